@@ -1,0 +1,243 @@
+/*
+ * pararnn.h - C ABI of the B200 (sm_100a) ParaRNN Newton-solve library
+ * (libpararnn.so).
+ *
+ * The library solves a whole nonlinear diagonal RNN recurrence in parallel
+ * over the sequence axis, the method of the page
+ *   "ParaRNN: Apple destrava treino paralelo de RNNs não-lineares e escala
+ *    pra 7B parâmetros" (cafecomtech.com, 2026-04-23):
+ *   - section "O compromisso que SSMs fizeram": the classic RNN applies
+ *     h_l = sigma(h_{l-1}, x_l) one step at a time; a linear SSM
+ *     h_l = A_l h_{l-1} + B_l x_l can instead be combined as a parallel
+ *     (associative) scan;
+ *   - section "A sacada: método de Newton": the whole sequence is one system
+ *     of equations whose unknowns are all hidden states; Newton linearises it
+ *     with the Jacobians, which take the place of A_l, so each iteration is a
+ *     linear SSM solved by a parallel scan;
+ *   - section "Engenharia pra escalar": with diagonal matrices in the cell
+ *     the Jacobian is diagonal (ParaGRU) or 2x2 block-diagonal per channel
+ *     over (c, h) (ParaLSTM), and Newton iterations, system assembly and
+ *     the parallel reduction run fused in one kernel.
+ *
+ * Cells (per channel d; s = logistic; the pages state only that the cell's
+ * matrices are diagonal, these are the diagonal GRU / LSTM):
+ *   GRU : z = s(u_z + a_z h), r = s(u_r + a_r h), c = tanh(u_c + a_c r h),
+ *         h' = (1 - z) h + z c                       gates u = (z, r, c)
+ *   LSTM: i = s(u_i + a_i h), f = s(u_f + a_f h), o = s(u_o + a_o h),
+ *         g = tanh(u_g + a_g h), c' = f c + i g, h' = o tanh(c')
+ *                                                    gates u = (i, f, o, g)
+ *
+ * Newton solve (reading of the pages, which leave these open):
+ *   unknowns H = (h_1..h_L) (and c_1..c_L), F_l(H) = state_l - cell(state_{l-1}, u_l);
+ *   initial guess H^0 = 0; r_k = max |F(H^k)| over all b, l, d and both LSTM
+ *   components; stop at the first k with r_k <= tol, or at k = max_iters;
+ *   iters = number of Newton updates in the returned states, residual = r of
+ *   the returned states.  Newton update: delta_l = J_l delta_{l-1} - F_l,
+ *   delta_0 = 0, H^{k+1} = H^k + delta, with J_l = d cell / d state_{l-1}
+ *   at H^k.
+ *
+ * Conventions for every entry point:
+ *   - Layouts are row-major with D fastest: u [B][L][G][D] (G = 3 or 4),
+ *     a [G][D], h0/c0 [B][D], states and gradients [B][L][D].
+ *   - All array pointers are DEVICE pointers, 16-byte aligned, owned by the
+ *     caller.  The library never allocates device memory; scratch space is
+ *     the caller's `workspace` (size from the *_workspace_size query,
+ *     256-byte aligned).  Inputs are never modified; outputs are fully
+ *     overwritten.
+ *   - B, L, D >= 1; D must be a multiple of 8 (else PARARNN_ERR_UNSUPPORTED);
+ *     B*L*D*4 bytes must fit in 2^40.  Violations return an error before any
+ *     work is queued.  Errors never abort the process; details are in
+ *     pararnn_last_error() (thread-local).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream) of the
+ *     current device.  Work is queued on it.
+ *   - Every wait inside the kernels is bounded (about 2 s); a wait that runs
+ *     out makes the call report PARARNN_ERR_TIMEOUT instead of hanging.
+ */
+#ifndef PARARNN_H
+#define PARARNN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PARARNN_API __attribute__((visibility("default")))
+#else
+#define PARARNN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PARARNN_OK = 0,
+    PARARNN_NOT_CONVERGED = 1,     /* warning: outputs valid, residual > tol  */
+    PARARNN_ERR_INVALID_ARG = -1,  /* bad pointer, size, tolerance, ...      */
+    PARARNN_ERR_WORKSPACE = -2,    /* workspace missing or too small         */
+    PARARNN_ERR_CUDA = -3,         /* a CUDA runtime call failed             */
+    PARARNN_ERR_TIMEOUT = -4,      /* a bounded device-side wait ran out     */
+    PARARNN_ERR_NONFINITE = -5,    /* residual is NaN or inf                 */
+    PARARNN_ERR_UNSUPPORTED = -6   /* e.g. D not a multiple of 8             */
+} pararnn_status;
+
+typedef enum { PARARNN_F32 = 0, PARARNN_BF16 = 1 } pararnn_dtype;
+
+/* ABI-identical to cudaStream_t. */
+typedef struct CUstream_st* pararnn_stream_t;
+
+/* Outcome of the last solve / adjoint run on a workspace (see
+ * pararnn_read_result). */
+typedef struct {
+    int32_t status;    /* pararnn_status                                    */
+    int32_t iters;     /* Newton updates applied to the returned states     */
+    float residual;    /* max |F| of the returned states                    */
+    float residual0;   /* max |F| of the initial guess H^0 = 0              */
+} pararnn_result;
+
+/* ----------------------------------------------------------- workspaces */
+
+/* Bytes of device workspace needed by the solves and adjoints for a given
+ * shape.  0 means the shape is invalid. */
+PARARNN_API size_t pararnn_gru_workspace_size(int64_t B, int64_t L, int64_t D);
+PARARNN_API size_t pararnn_lstm_workspace_size(int64_t B, int64_t L, int64_t D);
+PARARNN_API size_t pararnn_gru_adjoint_workspace_size(int64_t B, int64_t L, int64_t D);
+PARARNN_API size_t pararnn_lstm_adjoint_workspace_size(int64_t B, int64_t L, int64_t D);
+
+/* ---------------------------------------------------------------- solves */
+
+/* ParaGRU Newton solve ("A sacada: método de Newton"; diagonal Jacobian,
+ * "Engenharia pra escalar").  One cooperative kernel runs every Newton
+ * iteration: per iteration it evaluates the cell, its Jacobian and the
+ * residual at every (b, l, d), scans the affine maps (A_l, -F_l) over l,
+ * updates the states in place, and re-evaluates the residual of the new
+ * states to decide convergence on the device.
+ *   u        [B][L][3][D] gate pre-activations (z, r, c), dtype u_dtype
+ *   a        [3][D] fp32 diagonal recurrence weights (a_z, a_r, a_c)
+ *   h0       [B][D] fp32 initial state, or NULL for zeros
+ *   h        [B][L][D] fp32 output h_1..h_L
+ *   tol      >= 0, finite; max_iters >= 0
+ *   iters_out, residual_out: host pointers (may be NULL)
+ * Synchronous: returns after the stream has finished the solve.  Returns
+ * PARARNN_OK, PARARNN_NOT_CONVERGED (last iterate and its residual are
+ * returned), PARARNN_ERR_NONFINITE, or an error. */
+PARARNN_API pararnn_status pararnn_gru_solve(const void* u, pararnn_dtype u_dtype, const float* a,
+                                 const float* h0, float* h, int64_t B, int64_t L, int64_t D,
+                                 float tol, int max_iters, void* workspace,
+                                 size_t workspace_bytes, pararnn_stream_t stream,
+                                 int* iters_out, float* residual_out);
+
+/* Same as pararnn_gru_solve but only queues the work on `stream`; the outcome
+ * stays in the workspace until pararnn_read_result. */
+PARARNN_API pararnn_status pararnn_gru_solve_async(const void* u, pararnn_dtype u_dtype, const float* a,
+                                       const float* h0, float* h, int64_t B, int64_t L,
+                                       int64_t D, float tol, int max_iters, void* workspace,
+                                       size_t workspace_bytes, pararnn_stream_t stream);
+
+/* ParaLSTM Newton solve over the per-channel state (c, h) with the 2x2
+ * block-diagonal Jacobian ("Engenharia pra escalar").
+ *   u [B][L][4][D] gates (i, f, o, g); a [4][D]; c0, h0 [B][D] or NULL;
+ *   c, h [B][L][D] outputs.  Otherwise as pararnn_gru_solve. */
+PARARNN_API pararnn_status pararnn_lstm_solve(const void* u, pararnn_dtype u_dtype, const float* a,
+                                  const float* c0, const float* h0, float* c, float* h,
+                                  int64_t B, int64_t L, int64_t D, float tol, int max_iters,
+                                  void* workspace, size_t workspace_bytes,
+                                  pararnn_stream_t stream, int* iters_out, float* residual_out);
+
+PARARNN_API pararnn_status pararnn_lstm_solve_async(const void* u, pararnn_dtype u_dtype, const float* a,
+                                        const float* c0, const float* h0, float* c, float* h,
+                                        int64_t B, int64_t L, int64_t D, float tol,
+                                        int max_iters, void* workspace, size_t workspace_bytes,
+                                        pararnn_stream_t stream);
+
+/* Synchronises `stream` and reads the outcome of the last solve or adjoint
+ * queued on `workspace`.  Returns result->status (or an error if the read
+ * itself fails).  `result` is a host pointer. */
+PARARNN_API pararnn_status pararnn_read_result(const void* workspace, pararnn_stream_t stream,
+                                   pararnn_result* result);
+
+/* -------------------------------------------------------------- adjoints */
+
+/* Gradients of a loss through the converged ParaGRU states.  The pages do
+ * not describe training gradients; the reading here: at the solution
+ * F(H) = 0, dLoss/du = (dF/du)^T lambda with lambda solving the transposed
+ * Newton system, i.e. the reverse-time linear recurrence
+ *   lambda_l = dh_l + A_{l+1} lambda_{l+1},   lambda_L = dh_L,
+ * which is again a linear SSM, scanned in reverse with A_l^T (= A_l here).
+ *   h        [B][L][D] converged forward states (from pararnn_gru_solve)
+ *   dh       [B][L][D] fp32 upstream gradient dLoss/dh_l
+ *   du       [B][L][3][D] fp32 output dLoss/du
+ *   da       [3][D] fp32 output dLoss/da, summed over b and l (overwritten,
+ *            deterministic: fixed summation order)
+ *   dh0      [B][D] fp32 output dLoss/dh0, or NULL
+ * Asynchronous on `stream`; a device-side failure is reported by
+ * pararnn_read_result on the same workspace. */
+PARARNN_API pararnn_status pararnn_gru_adjoint(const void* u, pararnn_dtype u_dtype, const float* a,
+                                   const float* h0, const float* h, const float* dh, float* du,
+                                   float* da, float* dh0, int64_t B, int64_t L, int64_t D,
+                                   void* workspace, size_t workspace_bytes,
+                                   pararnn_stream_t stream);
+
+/* ParaLSTM adjoint: reverse-time scan of the 2x2 transposed Jacobians
+ *   lambda_l = (dc_l, dh_l) + J_{l+1}^T lambda_{l+1}.
+ *   c, h     [B][L][D] converged forward states
+ *   dh       [B][L][D] upstream dLoss/dh; dc [B][L][D] dLoss/dc or NULL (= 0)
+ *   du       [B][L][4][D], da [4][D], dc0 / dh0 [B][D] or NULL.            */
+PARARNN_API pararnn_status pararnn_lstm_adjoint(const void* u, pararnn_dtype u_dtype, const float* a,
+                                    const float* c0, const float* h0, const float* c,
+                                    const float* h, const float* dh, const float* dc, float* du,
+                                    float* da, float* dc0, float* dh0, int64_t B, int64_t L,
+                                    int64_t D, void* workspace, size_t workspace_bytes,
+                                    pararnn_stream_t stream);
+
+/* ------------------------------------------------------------- baselines */
+
+/* Naive sequential application ("O compromisso que SSMs fizeram": one step
+ * at a time): one GPU thread per (b, d) channel walks l = 1..L.  Same
+ * outputs as the solves (to rounding); asynchronous on `stream`. */
+PARARNN_API pararnn_status pararnn_gru_sequential(const void* u, pararnn_dtype u_dtype, const float* a,
+                                      const float* h0, float* h, int64_t B, int64_t L,
+                                      int64_t D, pararnn_stream_t stream);
+PARARNN_API pararnn_status pararnn_lstm_sequential(const void* u, pararnn_dtype u_dtype, const float* a,
+                                       const float* c0, const float* h0, float* c, float* h,
+                                       int64_t B, int64_t L, int64_t D,
+                                       pararnn_stream_t stream);
+
+/* Plain diagonal linear scan, the SSM of "O compromisso que SSMs fizeram",
+ * as a lower bound on one scan pass over the same [B][L][3][D] input: the
+ * GRU with zero recurrence weights,
+ *   h_l = (1 - s(u_z)) h_{l-1} + s(u_z) tanh(u_c),
+ * which reads two of the three gate streams.  One pass, no Newton;
+ * asynchronous on `stream`.  Workspace from
+ * pararnn_linear_scan_workspace_size. */
+PARARNN_API size_t pararnn_linear_scan_workspace_size(int64_t B, int64_t L, int64_t D);
+PARARNN_API pararnn_status pararnn_linear_scan(const void* u, pararnn_dtype u_dtype, const float* h0,
+                                   float* h, int64_t B, int64_t L, int64_t D, void* workspace,
+                                   size_t workspace_bytes, pararnn_stream_t stream);
+
+/* ------------------------------------------------------------ diagnostics */
+
+PARARNN_API const char* pararnn_status_string(pararnn_status s);
+/* Detail of the last error on the calling thread ("" if none). */
+PARARNN_API const char* pararnn_last_error(void);
+/* Library version as "major.minor.patch". */
+PARARNN_API const char* pararnn_version(void);
+/* Number of kernels this library has launched in this process (all threads). */
+PARARNN_API uint64_t pararnn_kernel_launch_count(void);
+
+/* Failure-detection self tests.  Each launches a small kernel that runs one
+ * of the library's bounded waits against a condition nothing will satisfy:
+ *   which = 0: the decoupled look-back of a tile whose predecessor never
+ *              publishes;
+ *   which = 1: the grid barrier (one CTA of a cooperative launch never
+ *              arrives).
+ * The wait must give up after `limit_ns` nanoseconds and the call must return
+ * PARARNN_ERR_TIMEOUT with the context still usable.  Needs a workspace of
+ * at least 16384 bytes.  Synchronous. */
+PARARNN_API pararnn_status pararnn_selftest_wait_timeout(int which, int64_t limit_ns, void* workspace,
+                                             size_t workspace_bytes, pararnn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARARNN_H */

@@ -1,0 +1,38 @@
+"""B200-native ParaRNN Newton solve (ParaGRU / ParaLSTM) behind a C ABI.
+
+The CUDA library ``libpararnn.so`` (built in-tree by ``build.py``) does all
+the work; ``capi`` is its thin ctypes binding, with the same entry-point
+names as ``include/pararnn.h``.  ``workloads`` draws the seeded synthetic
+inputs and needs no library.
+
+Binding names are resolved on first use; if the library is not built that
+first use raises ImportError (there is no fallback).
+"""
+import importlib
+
+__all__ = [
+    "PararnnError",
+    "pararnn_gru_adjoint",
+    "pararnn_gru_adjoint_workspace_size",
+    "pararnn_gru_sequential",
+    "pararnn_gru_solve",
+    "pararnn_gru_solve_async",
+    "pararnn_gru_workspace_size",
+    "pararnn_linear_scan",
+    "pararnn_linear_scan_workspace_size",
+    "pararnn_lstm_adjoint",
+    "pararnn_lstm_adjoint_workspace_size",
+    "pararnn_lstm_sequential",
+    "pararnn_lstm_solve",
+    "pararnn_lstm_solve_async",
+    "pararnn_lstm_workspace_size",
+    "pararnn_read_result",
+    "pararnn_selftest_wait_timeout",
+]
+
+
+def __getattr__(name):
+    if name in __all__ or name == "capi":
+        capi = importlib.import_module(".capi", __name__)
+        return capi if name == "capi" else getattr(capi, name)
+    raise AttributeError(name)

@@ -1,0 +1,365 @@
+"""Thin Python binding of libpararnn.so (ctypes).
+
+Argument marshalling only: every step of the solve, adjoint and baselines
+runs in the library's CUDA kernels.  PyTorch supplies device memory, streams
+and host<->device copies.  There is no CPU fallback: if the library is
+missing, importing this module raises ImportError.
+
+Names follow the C ABI in include/pararnn.h.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpararnn.so")
+
+OK = 0
+NOT_CONVERGED = 1
+ERR_INVALID_ARG = -1
+ERR_WORKSPACE = -2
+ERR_CUDA = -3
+ERR_TIMEOUT = -4
+ERR_NONFINITE = -5
+ERR_UNSUPPORTED = -6
+
+F32 = 0
+BF16 = 1
+
+
+class PararnnError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"pararnn status {status}: {msg}")
+        self.status = status
+
+
+class Result(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_int32), ("iters", ctypes.c_int32),
+                ("residual", ctypes.c_float), ("residual0", ctypes.c_float)]
+
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_st = ctypes.c_int
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "pararnn_gru_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "pararnn_lstm_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "pararnn_gru_adjoint_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "pararnn_lstm_adjoint_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "pararnn_linear_scan_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "pararnn_gru_solve": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int,
+                                _vp, ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_int),
+                                ctypes.POINTER(ctypes.c_float)]),
+    "pararnn_gru_solve_async": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float,
+                                      ctypes.c_int, _vp, ctypes.c_size_t, _vp]),
+    "pararnn_lstm_solve": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float,
+                                 ctypes.c_int, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_int),
+                                 ctypes.POINTER(ctypes.c_float)]),
+    "pararnn_lstm_solve_async": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                       ctypes.c_float, ctypes.c_int, _vp, ctypes.c_size_t, _vp]),
+    "pararnn_read_result": (_st, [_vp, _vp, ctypes.POINTER(Result)]),
+    "pararnn_gru_adjoint": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                  ctypes.c_size_t, _vp]),
+    "pararnn_lstm_adjoint": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
+    "pararnn_gru_sequential": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "pararnn_lstm_sequential": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "pararnn_linear_scan": (_st, [_vp, _st, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
+    "pararnn_status_string": (ctypes.c_char_p, [_st]),
+    "pararnn_last_error": (ctypes.c_char_p, []),
+    "pararnn_version": (ctypes.c_char_p, []),
+    "pararnn_kernel_launch_count": (ctypes.c_uint64, []),
+    "pararnn_selftest_wait_timeout": (_st, [ctypes.c_int, _i64, _vp, ctypes.c_size_t, _vp]),
+}
+
+
+def load(path=LIB_PATH):
+    """Load a build of the library and declare its signatures."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m nonlinear_rnn_newton_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = load()
+
+
+def last_error() -> str:
+    return lib.pararnn_last_error().decode()
+
+
+def status_string(s: int) -> str:
+    return lib.pararnn_status_string(int(s)).decode()
+
+
+def version() -> str:
+    return lib.pararnn_version().decode()
+
+
+def kernel_launch_count() -> int:
+    return int(lib.pararnn_kernel_launch_count())
+
+
+def _check(status, allow=(OK, NOT_CONVERGED, ERR_NONFINITE)):
+    if status not in allow:
+        raise PararnnError(status, f"{status_string(status)}: {last_error()}")
+    return status
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device, stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(u):
+    if u.dtype == torch.bfloat16:
+        return BF16
+    if u.dtype == torch.float32:
+        return F32
+    raise TypeError(f"u must be bfloat16 or float32, got {u.dtype}")
+
+
+def _need(t, name, shape, dtype=torch.float32, device=None):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, is on {t.device}")
+
+
+def _workspace(nbytes, device, workspace):
+    """The caller's workspace as is (the library checks its size), or a new one."""
+    if workspace is None:
+        return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    return workspace
+
+
+# ------------------------------------------------------------------ sizes
+
+def pararnn_gru_workspace_size(B, L, D):
+    return int(lib.pararnn_gru_workspace_size(B, L, D))
+
+
+def pararnn_lstm_workspace_size(B, L, D):
+    return int(lib.pararnn_lstm_workspace_size(B, L, D))
+
+
+def pararnn_gru_adjoint_workspace_size(B, L, D):
+    return int(lib.pararnn_gru_adjoint_workspace_size(B, L, D))
+
+
+def pararnn_lstm_adjoint_workspace_size(B, L, D):
+    return int(lib.pararnn_lstm_adjoint_workspace_size(B, L, D))
+
+
+def pararnn_linear_scan_workspace_size(B, L, D):
+    return int(lib.pararnn_linear_scan_workspace_size(B, L, D))
+
+
+# ------------------------------------------------------------------ solves
+
+def _to_device(t, device, stream):
+    if t is None or t.device == device:
+        return t
+    with torch.cuda.stream(stream):
+        return t.to(device, non_blocking=True)
+
+
+def pararnn_gru_solve(u, a, h0=None, tol=1e-6, max_iters=10, h=None, workspace=None, stream=None,
+                      device=None):
+    """ParaGRU Newton solve.  u [B,L,3,D] (bf16/fp32), a [3,D] fp32, h0 [B,D]
+    fp32 or None.  Returns (h [B,L,D], iters, residual, status).
+
+    Device tensors are used in place.  Host (CPU) tensors are copied to
+    ``device`` (default cuda:0) and the states copied back to the host."""
+    host = u.device.type == "cpu"
+    dev = torch.device(device or "cuda:0") if host else u.device
+    strm = stream or torch.cuda.current_stream(dev)
+    if host:
+        u, a, h0 = (_to_device(t, dev, strm) for t in (u, a, h0))
+    B, L, G, D = u.shape
+    if G != 3:
+        raise ValueError("GRU gates must be [B,L,3,D]")
+    _need(a, "a", (3, D), device=dev)
+    _need(h0, "h0", (B, D), device=dev)
+    dh = h if (h is not None and not host) else None
+    if dh is None:
+        dh = torch.empty((B, L, D), dtype=torch.float32, device=dev)
+    _need(dh, "h", (B, L, D), device=dev)
+    ws = _workspace(pararnn_gru_workspace_size(B, L, D), dev, workspace)
+    it = ctypes.c_int(0)
+    res = ctypes.c_float(0.0)
+    with torch.cuda.device(dev):
+        st = lib.pararnn_gru_solve(_ptr(u), _dtype_code(u), _ptr(a), _ptr(h0), _ptr(dh), B, L, D,
+                                   float(tol), int(max_iters), _ptr(ws), ws.numel(), _stream(dev, strm),
+                                   ctypes.byref(it), ctypes.byref(res))
+    _check(st)
+    if host:
+        out = h if h is not None else torch.empty((B, L, D), dtype=torch.float32, pin_memory=True)
+        out.copy_(dh)
+        dh = out
+    return dh, it.value, res.value, st
+
+
+def pararnn_gru_solve_async(u, a, h0, h, workspace, tol=1e-6, max_iters=10, stream=None):
+    """Queue a ParaGRU solve (device tensors only); read the outcome with
+    pararnn_read_result(workspace)."""
+    B, L, G, D = u.shape
+    st = lib.pararnn_gru_solve_async(_ptr(u), _dtype_code(u), _ptr(a), _ptr(h0), _ptr(h), B, L, D,
+                                     float(tol), int(max_iters), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(u.device, stream))
+    return _check(st)
+
+
+def pararnn_lstm_solve(u, a, c0=None, h0=None, tol=1e-6, max_iters=10, c=None, h=None, workspace=None,
+                       stream=None, device=None):
+    """ParaLSTM Newton solve.  u [B,L,4,D] gates (i,f,o,g).  Returns
+    (c, h, iters, residual, status).  Host tensors are handled as in
+    pararnn_gru_solve."""
+    host = u.device.type == "cpu"
+    dev = torch.device(device or "cuda:0") if host else u.device
+    strm = stream or torch.cuda.current_stream(dev)
+    if host:
+        u, a, c0, h0 = (_to_device(t, dev, strm) for t in (u, a, c0, h0))
+    B, L, G, D = u.shape
+    if G != 4:
+        raise ValueError("LSTM gates must be [B,L,4,D]")
+    _need(a, "a", (4, D), device=dev)
+    _need(c0, "c0", (B, D), device=dev)
+    _need(h0, "h0", (B, D), device=dev)
+    dc = c if (c is not None and not host) else torch.empty((B, L, D), dtype=torch.float32, device=dev)
+    dh = h if (h is not None and not host) else torch.empty((B, L, D), dtype=torch.float32, device=dev)
+    _need(dc, "c", (B, L, D), device=dev)
+    _need(dh, "h", (B, L, D), device=dev)
+    ws = _workspace(pararnn_lstm_workspace_size(B, L, D), dev, workspace)
+    it = ctypes.c_int(0)
+    res = ctypes.c_float(0.0)
+    with torch.cuda.device(dev):
+        st = lib.pararnn_lstm_solve(_ptr(u), _dtype_code(u), _ptr(a), _ptr(c0), _ptr(h0), _ptr(dc), _ptr(dh),
+                                    B, L, D, float(tol), int(max_iters), _ptr(ws), ws.numel(),
+                                    _stream(dev, strm), ctypes.byref(it), ctypes.byref(res))
+    _check(st)
+    if host:
+        oc = c if c is not None else torch.empty((B, L, D), dtype=torch.float32, pin_memory=True)
+        oh = h if h is not None else torch.empty((B, L, D), dtype=torch.float32, pin_memory=True)
+        oc.copy_(dc)
+        oh.copy_(dh)
+        dc, dh = oc, oh
+    return dc, dh, it.value, res.value, st
+
+
+def pararnn_lstm_solve_async(u, a, c0, h0, c, h, workspace, tol=1e-6, max_iters=10, stream=None):
+    B, L, G, D = u.shape
+    st = lib.pararnn_lstm_solve_async(_ptr(u), _dtype_code(u), _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h),
+                                      B, L, D, float(tol), int(max_iters), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(u.device, stream))
+    return _check(st)
+
+
+def pararnn_read_result(workspace, stream=None):
+    """Synchronise and return (status, iters, residual, residual0)."""
+    r = Result()
+    st = lib.pararnn_read_result(_ptr(workspace), _stream(workspace.device, stream), ctypes.byref(r))
+    if st in (ERR_INVALID_ARG, ERR_WORKSPACE, ERR_CUDA):
+        raise PararnnError(st, last_error())
+    return r.status, r.iters, r.residual, r.residual0
+
+
+# ---------------------------------------------------------------- adjoints
+
+def pararnn_gru_adjoint(u, a, h0, h, dh, du=None, da=None, dh0=None, want_dh0=True, workspace=None,
+                        stream=None):
+    """Gradients through the ParaGRU solution.  Returns (du [B,L,3,D], da [3,D], dh0 [B,D] or None).
+    Asynchronous on the stream."""
+    B, L, G, D = u.shape
+    dev = u.device
+    du = du if du is not None else torch.empty((B, L, 3, D), dtype=torch.float32, device=dev)
+    da = da if da is not None else torch.empty((3, D), dtype=torch.float32, device=dev)
+    if dh0 is None and want_dh0:
+        dh0 = torch.empty((B, D), dtype=torch.float32, device=dev)
+    for t, n, s in ((a, "a", (3, D)), (h0, "h0", (B, D)), (h, "h", (B, L, D)), (dh, "dh", (B, L, D)),
+                    (du, "du", (B, L, 3, D)), (da, "da", (3, D)), (dh0, "dh0", (B, D))):
+        _need(t, n, s, device=dev)
+    ws = _workspace(pararnn_gru_adjoint_workspace_size(B, L, D), dev, workspace)
+    st = lib.pararnn_gru_adjoint(_ptr(u), _dtype_code(u), _ptr(a), _ptr(h0), _ptr(h), _ptr(dh), _ptr(du),
+                                 _ptr(da), _ptr(dh0), B, L, D, _ptr(ws), ws.numel(), _stream(dev, stream))
+    _check(st, allow=(OK,))
+    return du, da, dh0
+
+
+def pararnn_lstm_adjoint(u, a, c0, h0, c, h, dh, dc=None, du=None, da=None, dc0=None, dh0=None,
+                         want_ds0=True, workspace=None, stream=None):
+    """Gradients through the ParaLSTM solution.  Returns (du [B,L,4,D], da [4,D], dc0, dh0)."""
+    B, L, G, D = u.shape
+    dev = u.device
+    du = du if du is not None else torch.empty((B, L, 4, D), dtype=torch.float32, device=dev)
+    da = da if da is not None else torch.empty((4, D), dtype=torch.float32, device=dev)
+    if want_ds0:
+        dc0 = dc0 if dc0 is not None else torch.empty((B, D), dtype=torch.float32, device=dev)
+        dh0 = dh0 if dh0 is not None else torch.empty((B, D), dtype=torch.float32, device=dev)
+    for t, n, s in ((a, "a", (4, D)), (c0, "c0", (B, D)), (h0, "h0", (B, D)), (c, "c", (B, L, D)),
+                    (h, "h", (B, L, D)), (dh, "dh", (B, L, D)), (dc, "dc", (B, L, D)),
+                    (du, "du", (B, L, 4, D)), (da, "da", (4, D)), (dc0, "dc0", (B, D)), (dh0, "dh0", (B, D))):
+        _need(t, n, s, device=dev)
+    ws = _workspace(pararnn_lstm_adjoint_workspace_size(B, L, D), dev, workspace)
+    st = lib.pararnn_lstm_adjoint(_ptr(u), _dtype_code(u), _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h),
+                                  _ptr(dh), _ptr(dc), _ptr(du), _ptr(da), _ptr(dc0), _ptr(dh0), B, L, D,
+                                  _ptr(ws), ws.numel(), _stream(dev, stream))
+    _check(st, allow=(OK,))
+    return du, da, dc0, dh0
+
+
+# --------------------------------------------------------------- baselines
+
+def pararnn_gru_sequential(u, a, h0=None, h=None, stream=None):
+    B, L, G, D = u.shape
+    h = h if h is not None else torch.empty((B, L, D), dtype=torch.float32, device=u.device)
+    st = lib.pararnn_gru_sequential(_ptr(u), _dtype_code(u), _ptr(a), _ptr(h0), _ptr(h), B, L, D,
+                                    _stream(u.device, stream))
+    _check(st, allow=(OK,))
+    return h
+
+
+def pararnn_lstm_sequential(u, a, c0=None, h0=None, c=None, h=None, stream=None):
+    B, L, G, D = u.shape
+    c = c if c is not None else torch.empty((B, L, D), dtype=torch.float32, device=u.device)
+    h = h if h is not None else torch.empty((B, L, D), dtype=torch.float32, device=u.device)
+    st = lib.pararnn_lstm_sequential(_ptr(u), _dtype_code(u), _ptr(a), _ptr(c0), _ptr(h0), _ptr(c), _ptr(h),
+                                     B, L, D, _stream(u.device, stream))
+    _check(st, allow=(OK,))
+    return c, h
+
+
+def pararnn_linear_scan(u, h0=None, h=None, workspace=None, stream=None):
+    B, L, G, D = u.shape
+    h = h if h is not None else torch.empty((B, L, D), dtype=torch.float32, device=u.device)
+    ws = _workspace(pararnn_linear_scan_workspace_size(B, L, D), u.device, workspace)
+    st = lib.pararnn_linear_scan(_ptr(u), _dtype_code(u), _ptr(h0), _ptr(h), B, L, D, _ptr(ws), ws.numel(),
+                                 _stream(u.device, stream))
+    _check(st, allow=(OK,))
+    return h
+
+
+def pararnn_selftest_wait_timeout(which, limit_ns, workspace, stream=None):
+    """Returns the status (ERR_TIMEOUT expected)."""
+    return int(lib.pararnn_selftest_wait_timeout(int(which), int(limit_ns), _ptr(workspace),
+                                                 workspace.numel(), _stream(workspace.device, stream)))

@@ -1,0 +1,713 @@
+// C ABI of libpararnn.so: argument checks, workspace layout, TMA descriptors
+// and kernel launches for the ParaRNN Newton solves, adjoints and baselines.
+// The entry points and their conventions are documented in include/pararnn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "pararnn.h"
+#include "pararnn_internal.h"
+#include "device_common.cuh"
+#include "cells.cuh"
+#include "newton.cuh"
+#include "sequential.cuh"
+#include "adjoint.cuh"
+#include "linear_scan.cuh"
+
+using namespace pararnn;
+
+namespace {
+
+thread_local char t_err[512] = "";
+std::atomic<unsigned long long> g_launches{0};
+
+pararnn_status fail(pararnn_status s, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_err, sizeof(t_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+#define CUDA_TRY(expr)                                                                        \
+    do {                                                                                      \
+        cudaError_t e_ = (expr);                                                              \
+        if (e_ != cudaSuccess)                                                                \
+            return fail(PARARNN_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));    \
+    } while (0)
+
+#define TRY(expr)                                 \
+    do {                                          \
+        pararnn_status s_ = (expr);               \
+        if (s_ != PARARNN_OK) return s_;          \
+    } while (0)
+
+// Timesteps per warp in a tile (a tile has 8 warps).  Compile-time tuning
+// knobs; the workspace layout follows them.
+#ifndef PARARNN_GRU_ROWS
+#define PARARNN_GRU_ROWS 4
+#endif
+#ifndef PARARNN_LSTM_ROWS
+#define PARARNN_LSTM_ROWS 2
+#endif
+#ifndef PARARNN_ADJ_ROWS
+#define PARARNN_ADJ_ROWS 4
+#endif
+#ifndef PARARNN_LIN_ROWS
+#define PARARNN_LIN_ROWS 8
+#endif
+constexpr size_t kSelftestWorkspace = 16384;
+constexpr int kLcGru = kWarps * PARARNN_GRU_ROWS;    // GRU solve
+constexpr int kLcLstm = kWarps * PARARNN_LSTM_ROWS;  // LSTM solve
+constexpr int kLcAdj = kWarps * PARARNN_ADJ_ROWS;    // adjoints
+constexpr int kLcLin = kWarps * PARARNN_LIN_ROWS;    // linear scan
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Shape {
+    long long B, L, D;
+    int S, n_chunks, n_tiles, Lc;
+};
+
+bool shape_ok(long long B, long long L, long long D) { return B >= 1 && L >= 1 && D >= 1; }
+
+pararnn_status make_shape(long long B, long long L, long long D, int Lc, Shape* s)
+{
+    if (!shape_ok(B, L, D)) return fail(PARARNN_ERR_INVALID_ARG, "B, L, D must be >= 1 (got %lld, %lld, %lld)", B, L, D);
+    if (D % 8 != 0) return fail(PARARNN_ERR_UNSUPPORTED, "D must be a multiple of 8 (got %lld)", D);
+    if (L > INT_MAX / 2 || B > INT_MAX / 2 || D > INT_MAX / 2)
+        return fail(PARARNN_ERR_INVALID_ARG, "dimension too large");
+    if ((double)B * (double)L * (double)D * 16.0 >= 1099511627776.0)
+        return fail(PARARNN_ERR_INVALID_ARG, "B*L*D too large (gate strides must stay below 2^40 bytes)");
+    s->B = B;
+    s->L = L;
+    s->D = D;
+    s->Lc = Lc;
+    s->S = int((D + kDc - 1) / kDc);
+    s->n_chunks = int((L + Lc - 1) / Lc);
+    const long long nt = (long long)s->n_chunks * B * s->S;
+    if (nt > INT_MAX / 4) return fail(PARARNN_ERR_INVALID_ARG, "too many tiles");
+    s->n_tiles = int(nt);
+    return PARARNN_OK;
+}
+
+struct ScanLayout {
+    size_t desc, extra, total;
+};
+
+// header | tile descriptors (tagged 64-bit words) | extra (boundary / partial
+// sums).  Header and descriptors are zeroed before every launch.
+ScanLayout scan_layout(const Shape& s, int desc_words, size_t extra_bytes)
+{
+    ScanLayout ly;
+    ly.desc = sizeof(WsHeader);
+    ly.extra = align256(ly.desc + size_t(s.n_tiles) * desc_words * 8);
+    ly.total = align256(ly.extra + extra_bytes);
+    return ly;
+}
+
+size_t solve_bnd_bytes(const Shape& s, int NS)
+{
+    return size_t(2) * NS * s.B * s.n_chunks * s.S * kDc * 4;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pararnn_status check_ptr(const void* p, const char* name, bool required)
+{
+    if (!p) return required ? fail(PARARNN_ERR_INVALID_ARG, "%s is NULL", name) : PARARNN_OK;
+    if (!aligned16(p)) return fail(PARARNN_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return PARARNN_OK;
+}
+
+pararnn_status check_dtype(pararnn_dtype dt)
+{
+    if (dt != PARARNN_F32 && dt != PARARNN_BF16) return fail(PARARNN_ERR_INVALID_ARG, "unknown u dtype %d", int(dt));
+    return PARARNN_OK;
+}
+
+pararnn_status check_workspace(const void* ws, size_t bytes, size_t need)
+{
+    if (!ws) return fail(PARARNN_ERR_WORKSPACE, "workspace is NULL");
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(PARARNN_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+    if (bytes < need) return fail(PARARNN_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", bytes, need);
+    return PARARNN_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Gate tensor [B][L][G][D] -> box [1][rows][G][kDc] (or a single gate g_box = 1).
+pararnn_status map_gates(CUtensorMap* m, const void* u, pararnn_dtype dt, int G, int g_box, const Shape& s,
+                         int rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t es = dt == PARARNN_BF16 ? 2 : 4;
+    cuuint64_t dims[4] = {cuuint64_t(s.D), cuuint64_t(G), cuuint64_t(s.L), cuuint64_t(s.B)};
+    cuuint64_t strides[3] = {cuuint64_t(s.D) * es, cuuint64_t(G) * s.D * es, cuuint64_t(s.L) * G * s.D * es};
+    cuuint32_t box[4] = {cuuint32_t(kDc), cuuint32_t(g_box), cuuint32_t(rows), 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    CUresult r = enc(m, dt == PARARNN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                     const_cast<void*>(u), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled(gates) failed: %d", int(r));
+    return PARARNN_OK;
+}
+
+// State tensor [B][L][D] fp32 -> box [1][rows][kDc].
+pararnn_status map_state(CUtensorMap* m, const float* x, const Shape& s, int rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {cuuint64_t(s.D), cuuint64_t(s.L), cuuint64_t(s.B)};
+    cuuint64_t strides[2] = {cuuint64_t(s.D) * 4, cuuint64_t(s.L) * s.D * 4};
+    cuuint32_t box[3] = {cuuint32_t(kDc), cuuint32_t(rows), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled(state) failed: %d", int(r));
+    return PARARNN_OK;
+}
+
+pararnn_status device_info(int* sms)
+{
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    CUDA_TRY(cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev));
+    int coop = 0;
+    CUDA_TRY(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
+    if (!coop) return fail(PARARNN_ERR_UNSUPPORTED, "device does not support cooperative launch");
+    return PARARNN_OK;
+}
+
+template <class K>
+pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid)
+{
+    int sms = 0;
+    TRY(device_info(&sms));
+    CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(smem)));
+    int occ = 0;
+    CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem));
+    if (occ < 1) return fail(PARARNN_ERR_CUDA, "kernel does not fit on an SM (smem %zu)", smem);
+    *grid = std::max(1, std::min(n_tiles, occ * sms));
+    return PARARNN_OK;
+}
+
+// ----------------------------------------------------------------- solves
+
+template <class Cell, class UT, int T>
+pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
+                             float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream)
+{
+    using LY = NewtonLayout<Cell, UT, T>;
+    constexpr int NS = Cell::NS;
+    const ScanLayout ly = scan_layout(s, LY::desc_words, solve_bnd_bytes(s, NS));
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));  // header + descriptors
+
+    CUtensorMap tu, t0, t1;
+    TRY(map_gates(&tu, u, dt, Cell::G, Cell::G, s, LY::Lc));
+    TRY(map_state(&t0, st[0], s, LY::Lc));
+    TRY(map_state(&t1, st[NS - 1], s, LY::Lc));
+
+    NewtonParams p;
+    p.a = a;
+    p.s0[0] = s0[0];
+    p.s0[1] = s0[1];
+    p.st[0] = st[0];
+    p.st[1] = st[1];
+    p.B = s.B;
+    p.L = s.L;
+    p.D = s.D;
+    p.S = s.S;
+    p.n_chunks = s.n_chunks;
+    p.n_tiles = s.n_tiles;
+    p.tol = tol;
+    p.max_iters = max_iters;
+    p.hdr = reinterpret_cast<WsHeader*>(wsb);
+    p.desc = reinterpret_cast<unsigned long long*>(wsb + ly.desc);
+    p.bnd = reinterpret_cast<float*>(wsb + ly.extra);
+    p.wait_ns = kWaitLimitNs;
+
+    auto kern = newton_solve_kernel<Cell, UT, T>;
+    int grid = 0;
+    TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid));
+    void* args[] = {(void*)&tu, (void*)&t0, (void*)&t1, (void*)&p};
+    CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(kThreads), args,
+                                         LY::smem_bytes, stream));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
+size_t solve_ws_bytes(int cell, long long B, long long L, long long D)
+{
+    if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
+    Shape s;
+    char saved[sizeof(t_err)];
+    memcpy(saved, t_err, sizeof(t_err));
+    pararnn_status st = make_shape(B, L, D, cell == 0 ? kLcGru : kLcLstm, &s);
+    memcpy(t_err, saved, sizeof(t_err));
+    if (st != PARARNN_OK) return 0;
+    if (cell == 0) return scan_layout(s, NewtonLayout<GruCell, float, kLcGru / kWarps>::desc_words, solve_bnd_bytes(s, 1)).total;
+    return scan_layout(s, NewtonLayout<LstmCell, float, kLcLstm / kWarps>::desc_words, solve_bnd_bytes(s, 2)).total;
+}
+
+pararnn_status solve_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* c0, const float* h0,
+                           float* c, float* h, long long B, long long L, long long D, float tol, int max_iters,
+                           void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(dt));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(h0, "h0", false));
+    TRY(check_ptr(h, "h", true));
+    if (cell == 1) {
+        TRY(check_ptr(c0, "c0", false));
+        TRY(check_ptr(c, "c", true));
+    }
+    if (!(tol >= 0.0f) || !std::isfinite(tol)) return fail(PARARNN_ERR_INVALID_ARG, "tol must be finite and >= 0");
+    if (max_iters < 0) return fail(PARARNN_ERR_INVALID_ARG, "max_iters must be >= 0");
+    Shape s;
+    TRY(make_shape(B, L, D, cell == 0 ? kLcGru : kLcLstm, &s));
+    TRY(check_workspace(ws, ws_bytes, solve_ws_bytes(cell, B, L, D)));
+    if (cell == 0) {
+        const float* s0[2] = {h0, nullptr};
+        float* st[2] = {h, nullptr};
+        if (dt == PARARNN_BF16)
+            return launch_newton<GruCell, uint16_t, kLcGru / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+        return launch_newton<GruCell, float, kLcGru / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+    }
+    const float* s0[2] = {c0, h0};
+    float* st[2] = {c, h};
+    if (dt == PARARNN_BF16)
+        return launch_newton<LstmCell, uint16_t, kLcLstm / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+    return launch_newton<LstmCell, float, kLcLstm / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+}
+
+pararnn_status read_header(const void* ws, cudaStream_t stream, WsHeader* h)
+{
+    if (!ws) return fail(PARARNN_ERR_WORKSPACE, "workspace is NULL");
+    CUDA_TRY(cudaMemcpyAsync(h, ws, sizeof(WsHeader), cudaMemcpyDeviceToHost, stream));
+    CUDA_TRY(cudaStreamSynchronize(stream));
+    return PARARNN_OK;
+}
+
+pararnn_status finish_sync(void* ws, cudaStream_t stream, int* iters_out, float* residual_out)
+{
+    pararnn_result r;
+    pararnn_status st = pararnn_read_result(ws, stream, &r);
+    if (st < 0 && st != PARARNN_ERR_NONFINITE) return st;
+    if (iters_out) *iters_out = r.iters;
+    if (residual_out) *residual_out = r.residual;
+    return st;
+}
+
+// --------------------------------------------------------------- adjoints
+
+size_t adjoint_ws_bytes(int cell, long long B, long long L, long long D)
+{
+    if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
+    Shape s;
+    char saved[sizeof(t_err)];
+    memcpy(saved, t_err, sizeof(t_err));
+    pararnn_status st = make_shape(B, L, D, kLcAdj, &s);
+    memcpy(t_err, saved, sizeof(t_err));
+    if (st != PARARNN_OK) return 0;
+    const int G = cell == 0 ? 3 : 4;
+    const int desc = cell == 0 ? AdjointLayout<GruCell, float, kLcAdj / kWarps>::desc_words
+                               : AdjointLayout<LstmCell, float, kLcAdj / kWarps>::desc_words;
+    return scan_layout(s, desc, size_t(s.n_tiles) * G * kDc * 4).total;
+}
+
+template <class Cell, class UT, int T>
+pararnn_status launch_adjoint(const Shape& s, const void* u, pararnn_dtype dt, const float* a,
+                              const float* const s0[2], const float* const st[2], const float* const g[2],
+                              float* du, float* da, float* const ds0[2], void* ws, cudaStream_t stream)
+{
+    using LY = AdjointLayout<Cell, UT, T>;
+    constexpr int NS = Cell::NS, G = Cell::G;
+    const ScanLayout ly = scan_layout(s, LY::desc_words, size_t(s.n_tiles) * G * kDc * 4);
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));
+
+    CUtensorMap tu, t0, t1, tg0, tg1;
+    TRY(map_gates(&tu, u, dt, G, G, s, LY::Lc));
+    TRY(map_state(&t0, st[0], s, LY::Lc));
+    TRY(map_state(&t1, st[NS - 1], s, LY::Lc));
+    const float* gfirst = g[0] ? g[0] : g[NS - 1];
+    TRY(map_state(&tg0, gfirst, s, LY::Lc));
+    TRY(map_state(&tg1, g[NS - 1], s, LY::Lc));
+
+    AdjointParams p;
+    p.a = a;
+    p.s0[0] = s0[0];
+    p.s0[1] = s0[1];
+    p.st[0] = st[0];
+    p.st[1] = st[1];
+    p.du = du;
+    p.ds0[0] = ds0[0];
+    p.ds0[1] = ds0[1];
+    p.B = s.B;
+    p.L = s.L;
+    p.D = s.D;
+    p.S = s.S;
+    p.n_chunks = s.n_chunks;
+    p.n_tiles = s.n_tiles;
+    p.has_g[0] = g[0] != nullptr;
+    p.has_g[1] = g[1] != nullptr;
+    p.hdr = reinterpret_cast<WsHeader*>(wsb);
+    p.desc = reinterpret_cast<unsigned long long*>(wsb + ly.desc);
+    p.partial = reinterpret_cast<float*>(wsb + ly.extra);
+    p.wait_ns = kWaitLimitNs;
+
+    auto kern = adjoint_kernel<Cell, UT, T>;
+    int grid = 0;
+    TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid));
+    kern<<<grid, kThreads, LY::smem_bytes, stream>>>(tu, t0, t1, tg0, tg1, p);
+    CUDA_TRY(cudaGetLastError());
+    const long long GD = (long long)G * s.D;
+    da_reduce_kernel<<<unsigned((GD + 31) / 32), 256, 0, stream>>>(p.partial, da, int(s.B) * s.n_chunks, s.S, G, s.D);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(2, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
+pararnn_status adjoint_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* c0,
+                             const float* h0, const float* c, const float* h, const float* dc, const float* dh,
+                             float* du, float* da, float* dc0, float* dh0, long long B, long long L, long long D,
+                             void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(dt));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(h0, "h0", false));
+    TRY(check_ptr(h, "h", true));
+    TRY(check_ptr(dh, "dh", true));
+    TRY(check_ptr(du, "du", true));
+    TRY(check_ptr(da, "da", true));
+    TRY(check_ptr(dh0, "dh0", false));
+    if (cell == 1) {
+        TRY(check_ptr(c0, "c0", false));
+        TRY(check_ptr(c, "c", true));
+        TRY(check_ptr(dc, "dc", false));
+        TRY(check_ptr(dc0, "dc0", false));
+    }
+    Shape s;
+    TRY(make_shape(B, L, D, kLcAdj, &s));
+    TRY(check_workspace(ws, ws_bytes, adjoint_ws_bytes(cell, B, L, D)));
+    if (cell == 0) {
+        const float* s0[2] = {h0, nullptr};
+        const float* st[2] = {h, nullptr};
+        const float* g[2] = {dh, nullptr};
+        float* ds0[2] = {dh0, nullptr};
+        if (dt == PARARNN_BF16)
+            return launch_adjoint<GruCell, uint16_t, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+        return launch_adjoint<GruCell, float, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+    }
+    const float* s0[2] = {c0, h0};
+    const float* st[2] = {c, h};
+    const float* g[2] = {dc, dh};
+    float* ds0[2] = {dc0, dh0};
+    if (dt == PARARNN_BF16)
+        return launch_adjoint<LstmCell, uint16_t, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+    return launch_adjoint<LstmCell, float, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+}
+
+// ------------------------------------------------------------ linear scan
+
+size_t linear_scan_ws_bytes(long long B, long long L, long long D)
+{
+    if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
+    Shape s;
+    char saved[sizeof(t_err)];
+    memcpy(saved, t_err, sizeof(t_err));
+    pararnn_status st = make_shape(B, L, D, kLcLin, &s);
+    memcpy(t_err, saved, sizeof(t_err));
+    if (st != PARARNN_OK) return 0;
+    return scan_layout(s, LinScanLayout<float, kLcLin / kWarps>::desc_words, 0).total;
+}
+
+template <class UT, int T>
+pararnn_status launch_linear_scan(const Shape& s, const void* u, pararnn_dtype dt, const float* h0, float* h, void* ws,
+                                  cudaStream_t stream)
+{
+    using LY = LinScanLayout<UT, T>;
+    const ScanLayout ly = scan_layout(s, LY::desc_words, 0);
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));
+    CUtensorMap tu1;
+    TRY(map_gates(&tu1, u, dt, 3, 1, s, LY::Lc));
+    LinScanParams p;
+    p.h0 = h0;
+    p.h = h;
+    p.B = s.B;
+    p.L = s.L;
+    p.D = s.D;
+    p.S = s.S;
+    p.n_chunks = s.n_chunks;
+    p.n_tiles = s.n_tiles;
+    p.hdr = reinterpret_cast<WsHeader*>(wsb);
+    p.desc = reinterpret_cast<unsigned long long*>(wsb + ly.desc);
+    p.wait_ns = kWaitLimitNs;
+    auto kern = linear_scan_kernel<UT, T>;
+    int grid = 0;
+    TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid));
+    kern<<<grid, kThreads, LY::smem_bytes, stream>>>(tu1, p);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
+pararnn_status linear_scan_async(const void* u, pararnn_dtype dt, const float* h0, float* h, long long B, long long L,
+                                 long long D, void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(dt));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(h0, "h0", false));
+    TRY(check_ptr(h, "h", true));
+    Shape s;
+    TRY(make_shape(B, L, D, kLcLin, &s));
+    TRY(check_workspace(ws, ws_bytes, linear_scan_ws_bytes(B, L, D)));
+    if (dt == PARARNN_BF16) return launch_linear_scan<uint16_t, kLcLin / kWarps>(s, u, dt, h0, h, ws, stream);
+    return launch_linear_scan<float, kLcLin / kWarps>(s, u, dt, h0, h, ws, stream);
+}
+
+// -------------------------------------------------------------- self tests
+
+pararnn_status selftest_wait_timeout(int which, long long limit_ns, void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    if (which != 0 && which != 1) return fail(PARARNN_ERR_INVALID_ARG, "which must be 0 or 1");
+    if (limit_ns <= 0 || limit_ns > 10000000000ll) return fail(PARARNN_ERR_INVALID_ARG, "limit_ns out of range");
+    TRY(check_workspace(ws, ws_bytes, kSelftestWorkspace));
+    CUDA_TRY(cudaMemsetAsync(ws, 0, kSelftestWorkspace, stream));
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+    unsigned long long* desc = reinterpret_cast<unsigned long long*>(wsb + sizeof(WsHeader));
+    unsigned long long lim = (unsigned long long)limit_ns;
+    if (which == 0) {
+        selftest_lookback_kernel<<<1, 32, 0, stream>>>(desc, &hdr->error, lim);
+        CUDA_TRY(cudaGetLastError());
+    } else {
+        int sms = 0;
+        TRY(device_info(&sms));
+        unsigned* counter = &hdr->bar;
+        int* err = &hdr->error;
+        void* args[] = {(void*)&counter, (void*)&err, (void*)&lim};
+        CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(selftest_barrier_kernel), dim3(2), dim3(32),
+                                             args, 0, stream));
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    WsHeader h;
+    TRY(read_header(ws, stream, &h));
+    if (h.error != 0) return fail(pararnn_status(h.error), "bounded wait gave up as expected");
+    return PARARNN_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+size_t pararnn_gru_workspace_size(int64_t B, int64_t L, int64_t D) { return solve_ws_bytes(0, B, L, D); }
+size_t pararnn_lstm_workspace_size(int64_t B, int64_t L, int64_t D) { return solve_ws_bytes(1, B, L, D); }
+
+pararnn_status pararnn_gru_solve_async(const void* u, pararnn_dtype u_dtype, const float* a, const float* h0, float* h,
+                                       int64_t B, int64_t L, int64_t D, float tol, int max_iters, void* workspace,
+                                       size_t workspace_bytes, pararnn_stream_t stream)
+{
+    return solve_async(0, u, u_dtype, a, nullptr, h0, nullptr, h, B, L, D, tol, max_iters, workspace,
+                       workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_gru_solve(const void* u, pararnn_dtype u_dtype, const float* a, const float* h0, float* h,
+                                 int64_t B, int64_t L, int64_t D, float tol, int max_iters, void* workspace,
+                                 size_t workspace_bytes, pararnn_stream_t stream, int* iters_out, float* residual_out)
+{
+    TRY(pararnn_gru_solve_async(u, u_dtype, a, h0, h, B, L, D, tol, max_iters, workspace, workspace_bytes, stream));
+    return finish_sync(workspace, reinterpret_cast<cudaStream_t>(stream), iters_out, residual_out);
+}
+
+pararnn_status pararnn_lstm_solve_async(const void* u, pararnn_dtype u_dtype, const float* a, const float* c0,
+                                        const float* h0, float* c, float* h, int64_t B, int64_t L, int64_t D,
+                                        float tol, int max_iters, void* workspace, size_t workspace_bytes,
+                                        pararnn_stream_t stream)
+{
+    return solve_async(1, u, u_dtype, a, c0, h0, c, h, B, L, D, tol, max_iters, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_lstm_solve(const void* u, pararnn_dtype u_dtype, const float* a, const float* c0,
+                                  const float* h0, float* c, float* h, int64_t B, int64_t L, int64_t D, float tol,
+                                  int max_iters, void* workspace, size_t workspace_bytes, pararnn_stream_t stream,
+                                  int* iters_out, float* residual_out)
+{
+    TRY(pararnn_lstm_solve_async(u, u_dtype, a, c0, h0, c, h, B, L, D, tol, max_iters, workspace, workspace_bytes,
+                                 stream));
+    return finish_sync(workspace, reinterpret_cast<cudaStream_t>(stream), iters_out, residual_out);
+}
+
+pararnn_status pararnn_read_result(const void* workspace, pararnn_stream_t stream, pararnn_result* result)
+{
+    WsHeader h;
+    TRY(read_header(workspace, reinterpret_cast<cudaStream_t>(stream), &h));
+    pararnn_result r = h.result;
+    if (h.error != 0) {
+        r.status = h.error;
+        fail(pararnn_status(h.error), "device-side error %d (%s)", h.error, pararnn_status_string(pararnn_status(h.error)));
+    }
+    if (result) *result = r;
+    return pararnn_status(r.status);
+}
+
+// ------------------------------------------------------------- adjoints
+
+size_t pararnn_gru_adjoint_workspace_size(int64_t B, int64_t L, int64_t D) { return adjoint_ws_bytes(0, B, L, D); }
+size_t pararnn_lstm_adjoint_workspace_size(int64_t B, int64_t L, int64_t D) { return adjoint_ws_bytes(1, B, L, D); }
+
+pararnn_status pararnn_gru_adjoint(const void* u, pararnn_dtype u_dtype, const float* a, const float* h0,
+                                   const float* h, const float* dh, float* du, float* da, float* dh0, int64_t B,
+                                   int64_t L, int64_t D, void* workspace, size_t workspace_bytes,
+                                   pararnn_stream_t stream)
+{
+    return adjoint_async(0, u, u_dtype, a, nullptr, h0, nullptr, h, nullptr, dh, du, da, nullptr, dh0, B, L, D,
+                         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_lstm_adjoint(const void* u, pararnn_dtype u_dtype, const float* a, const float* c0,
+                                    const float* h0, const float* c, const float* h, const float* dh, const float* dc,
+                                    float* du, float* da, float* dc0, float* dh0, int64_t B, int64_t L, int64_t D,
+                                    void* workspace, size_t workspace_bytes, pararnn_stream_t stream)
+{
+    return adjoint_async(1, u, u_dtype, a, c0, h0, c, h, dc, dh, du, da, dc0, dh0, B, L, D, workspace,
+                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------- baselines
+
+pararnn_status pararnn_gru_sequential(const void* u, pararnn_dtype u_dtype, const float* a, const float* h0, float* h,
+                                      int64_t B, int64_t L, int64_t D, pararnn_stream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(u_dtype));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(h0, "h0", false));
+    TRY(check_ptr(h, "h", true));
+    Shape s;
+    TRY(make_shape(B, L, D, 1, &s));
+    const long long n = B * D;
+    const dim3 grid(unsigned((n + 63) / 64)), block(64);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (u_dtype == PARARNN_BF16)
+        sequential_kernel<GruCell, uint16_t><<<grid, block, 0, st>>>(static_cast<const uint16_t*>(u), a, h0, nullptr,
+                                                                     h, nullptr, B, L, D);
+    else
+        sequential_kernel<GruCell, float><<<grid, block, 0, st>>>(static_cast<const float*>(u), a, h0, nullptr, h,
+                                                                  nullptr, B, L, D);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
+pararnn_status pararnn_lstm_sequential(const void* u, pararnn_dtype u_dtype, const float* a, const float* c0,
+                                       const float* h0, float* c, float* h, int64_t B, int64_t L, int64_t D,
+                                       pararnn_stream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(u_dtype));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(c0, "c0", false));
+    TRY(check_ptr(h0, "h0", false));
+    TRY(check_ptr(c, "c", true));
+    TRY(check_ptr(h, "h", true));
+    Shape s;
+    TRY(make_shape(B, L, D, 1, &s));
+    const long long n = B * D;
+    const dim3 grid(unsigned((n + 63) / 64)), block(64);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (u_dtype == PARARNN_BF16)
+        sequential_kernel<LstmCell, uint16_t><<<grid, block, 0, st>>>(static_cast<const uint16_t*>(u), a, c0, h0, c,
+                                                                      h, B, L, D);
+    else
+        sequential_kernel<LstmCell, float><<<grid, block, 0, st>>>(static_cast<const float*>(u), a, c0, h0, c, h, B,
+                                                                   L, D);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
+size_t pararnn_linear_scan_workspace_size(int64_t B, int64_t L, int64_t D) { return linear_scan_ws_bytes(B, L, D); }
+
+pararnn_status pararnn_linear_scan(const void* u, pararnn_dtype u_dtype, const float* h0, float* h, int64_t B,
+                                   int64_t L, int64_t D, void* workspace, size_t workspace_bytes,
+                                   pararnn_stream_t stream)
+{
+    return linear_scan_async(u, u_dtype, h0, h, B, L, D, workspace, workspace_bytes,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ----------------------------------------------------------- diagnostics
+
+const char* pararnn_status_string(pararnn_status s)
+{
+    switch (s) {
+    case PARARNN_OK: return "ok";
+    case PARARNN_NOT_CONVERGED: return "not converged";
+    case PARARNN_ERR_INVALID_ARG: return "invalid argument";
+    case PARARNN_ERR_WORKSPACE: return "workspace missing or too small";
+    case PARARNN_ERR_CUDA: return "CUDA error";
+    case PARARNN_ERR_TIMEOUT: return "device-side wait timed out";
+    case PARARNN_ERR_NONFINITE: return "non-finite residual";
+    case PARARNN_ERR_UNSUPPORTED: return "unsupported";
+    }
+    return "unknown status";
+}
+
+const char* pararnn_last_error(void) { return t_err; }
+
+const char* pararnn_version(void) { return "0.1.0"; }
+
+uint64_t pararnn_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+pararnn_status pararnn_selftest_wait_timeout(int which, int64_t limit_ns, void* workspace, size_t workspace_bytes,
+                                             pararnn_stream_t stream)
+{
+    return selftest_wait_timeout(which, limit_ns, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,41 @@
+// Internal constants and the device-side workspace header shared by the host
+// launcher and the kernels.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pararnn.h"
+
+namespace pararnn {
+
+#ifndef PARARNN_WARPS
+#define PARARNN_WARPS 8
+#endif
+constexpr int kWarps = PARARNN_WARPS;  // warps per CTA: each owns T consecutive timesteps
+constexpr int kThreads = 32 * kWarps;  // threads per CTA
+#ifndef PARARNN_MINB
+#define PARARNN_MINB (16 / PARARNN_WARPS)
+#endif
+constexpr int kMinBlocks = PARARNN_MINB;  // CTAs per SM the kernels are register-budgeted for
+constexpr int kV = 4;              // channels per lane
+constexpr int kDc = 32 * kV;       // channels per tile (one per lane x kV)
+
+// Default limit for every device-side wait (look-back flags, grid barrier,
+// TMA completion).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// First 256 bytes of every workspace.  Zeroed by the host before each run.
+struct alignas(256) WsHeader {
+    unsigned tick[4];  // tile ticket counter per pass slot (pass k uses k % 3)
+    unsigned res[4];   // max |F| bits of the updated states per pass slot
+    unsigned res0;     // max |F| bits of the initial guess
+    unsigned bar;      // grid barrier arrivals (monotone)
+    int error;         // first device-side error (pararnn_status < 0), 0 if none
+    int passes;        // Newton passes run
+    pararnn_result result;
+    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result)];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
+
+}  // namespace pararnn

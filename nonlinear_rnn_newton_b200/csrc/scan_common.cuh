@@ -1,0 +1,263 @@
+// Chunked parallel scan of affine maps, shared by the Newton solve, the
+// adjoint and the linear-scan baseline.
+//
+// Page: "ParaRNN: Apple destrava treino paralelo de RNNs não-lineares e escala
+// pra 7B parâmetros", section "O compromisso que SSMs fizeram": a linear
+// recurrence is an associative combination, so it can be evaluated as a tree
+// (O(log L) depth) instead of step by step; section "A sacada: método de
+// Newton": every Newton iteration is such a linear recurrence.
+//
+// Three levels: (1) each thread folds its T timesteps serially in registers;
+// (2) a warp-shuffle scan combines the warps' segments of a tile, each
+// channel group handled by kWarps lanes; (3) a decoupled look-back combines tiles
+// across CTAs: every tile publishes its aggregate right away, then walks back
+// over predecessors' aggregates until it meets an inclusive prefix, and
+// publishes its own inclusive value.  Values travel as tagged 64-bit words
+// (each word is its own ready flag, so no fences); every wait is bounded.
+#pragma once
+
+#include "cells.cuh"
+
+namespace pararnn {
+
+constexpr int kScanPad = kDc + 4;  // padded scratch row (floats): conflict-free strided reads
+
+template <class Map>
+__device__ __forceinline__ Map shfl_up_map8(const Map& x, int delta)
+{
+    Map r;
+#pragma unroll
+    for (int i = 0; i < Map::kFloats; ++i) r.set(i, __shfl_up_sync(0xffffffffu, x.get(i), delta, kWarps));
+    return r;
+}
+
+// Write a thread's kV per-channel maps to segment position `pos` of the scratch
+// [NC][kWarps][kScanPad].
+template <class Map>
+__device__ __forceinline__ void scan_put(float* scan, int pos, int lane, const Map (&m)[kV])
+{
+#pragma unroll
+    for (int i = 0; i < Map::kFloats; ++i) {
+        float v4[kV];
+#pragma unroll
+        for (int j = 0; j < kV; ++j) v4[j] = m[j].get(i);
+        store4(scan + (i * kWarps + pos) * kScanPad + lane * kV, v4);
+    }
+}
+
+// Read one channel's map at segment position `pos`.
+template <class Map>
+__device__ __forceinline__ Map scan_get(const float* scan, int pos, int ch)
+{
+    Map m;
+#pragma unroll
+    for (int i = 0; i < Map::kFloats; ++i) m.set(i, scan[(i * kWarps + pos) * kScanPad + ch]);
+    return m;
+}
+
+// In-place exclusive scan over the kWarps segment positions of the scratch,
+// for all kDc channels; the full-tile aggregate goes to tagg [NC][kDc].
+// Called by all kThreads threads between two __syncthreads.
+template <class Map>
+__device__ __forceinline__ void cta_segment_scan(float* scan, float* tagg, int tid)
+{
+    constexpr int NC = Map::kFloats;
+    const int grp = tid / kWarps;  // channels grp*kV .. grp*kV+kV-1
+    const int seg = tid % kWarps;  // segment position
+    Map x[kV];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        F4 v = load4(scan + (i * kWarps + seg) * kScanPad + grp * kV);
+#pragma unroll
+        for (int j = 0; j < kV; ++j) x[j].set(i, v.v[j]);
+    }
+#pragma unroll
+    for (int off = 1; off < kWarps; off <<= 1) {
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+            Map y = shfl_up_map8(x[j], off);
+            if (seg >= off) x[j] = compose(x[j], y);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kV; ++j) {
+        Map y = shfl_up_map8(x[j], 1);
+        if (seg == 0) y = Map::identity();
+        if (seg == kWarps - 1) {
+#pragma unroll
+            for (int i = 0; i < NC; ++i) tagg[i * kDc + grp * kV + j] = x[j].get(i);
+        }
+        x[j] = y;
+    }
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        float v4[kV];
+#pragma unroll
+        for (int j = 0; j < kV; ++j) v4[j] = x[j].get(i);
+        store4(scan + (i * kWarps + seg) * kScanPad + grp * kV, v4);
+    }
+}
+
+// Published values are tagged 64-bit words: the float in the low half, a tag
+// in the high half.  An aligned 64-bit access is single-copy atomic, so a
+// reader that sees the expected tag also sees the value written with it: the
+// word is its own flag, and neither side needs a fence.  Tags are 2*epoch+1
+// (tile aggregate) and 2*epoch+2 (inclusive value); the words are zeroed
+// before each launch, and tags only grow within a launch.
+__device__ __forceinline__ unsigned long long tag_word(float v, unsigned tag)
+{
+    return (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+}
+
+__device__ __forceinline__ void st_words2(unsigned long long* p, unsigned long long a, unsigned long long b)
+{
+    asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+}
+
+__device__ __forceinline__ void ld_words2(const unsigned long long* p, unsigned long long& a, unsigned long long& b)
+{
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+
+// Descriptor of one tile in the workspace (tagged words):
+//   aggregates [32 lanes][kV * NC] then inclusive values [32 lanes][kV * NS].
+template <class Map, int NS>
+struct TileDesc {
+    static constexpr int agg_words = 32 * kV * Map::kFloats;
+    static constexpr int words = 32 * kV * (Map::kFloats + NS);
+};
+
+// Store n (even) tagged words.
+template <int N>
+__device__ __forceinline__ void publish_words(unsigned long long* dst, const float (&v)[N], unsigned tag)
+{
+    static_assert(N % 2 == 0, "pairs");
+#pragma unroll
+    for (int i = 0; i < N; i += 2) st_words2(dst + i, tag_word(v[i], tag), tag_word(v[i + 1], tag));
+}
+
+// Load n (even) words; true if every tag equals `tag`.
+template <int N>
+__device__ __forceinline__ bool fetch_words(const unsigned long long* src, float (&v)[N], unsigned tag)
+{
+    static_assert(N % 2 == 0, "pairs");
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < N; i += 2) {
+        unsigned long long a, b;
+        ld_words2(src + i, a, b);
+        ok = ok && unsigned(a >> 32) == tag && unsigned(b >> 32) == tag;
+        v[i] = __uint_as_float(unsigned(a));
+        v[i + 1] = __uint_as_float(unsigned(b));
+    }
+    return ok;
+}
+
+// Decoupled look-back, run by one full warp; lane owns channels lane*kV..+kV-1.
+//   ticket:    this tile's ticket; its predecessor is ticket - stride
+//   has_pred:  false for the first tile of a sequence (carry = `init`)
+//   epoch:     tags 2*epoch+1 (aggregate), 2*epoch+2 (inclusive)
+//   ta:        this tile's aggregate maps
+//   carry:     out: value entering this tile (the predecessors' inclusive)
+// Publishes the aggregate (if there is a predecessor) and, once the carry is
+// known, the inclusive value apply(ta, carry).  Each lane walks back on its
+// own; a wait that runs out of time raises PARARNN_ERR_TIMEOUT and returns
+// false.
+template <class Map, int NS>
+__device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, int epoch, const Map (&ta)[kV],
+                                         const float (&init)[NS][kV], float (&carry)[NS][kV],
+                                         unsigned long long* desc, int lane, int* err,
+                                         unsigned long long wait_ns)
+{
+    using TD = TileDesc<Map, NS>;
+    constexpr int NC = Map::kFloats;
+    const unsigned t_agg = 2u * epoch + 1u, t_incl = 2u * epoch + 2u;
+    unsigned long long* mine = desc + (size_t)ticket * TD::words;
+#pragma unroll
+    for (int q = 0; q < NS; ++q)
+#pragma unroll
+        for (int j = 0; j < kV; ++j) carry[q][j] = init[q][j];
+    bool ok = true;
+    if (has_pred) {
+        {
+            float av[kV * NC];
+#pragma unroll
+            for (int j = 0; j < kV; ++j)
+#pragma unroll
+                for (int i = 0; i < NC; ++i) av[j * NC + i] = ta[j].get(i);
+            publish_words(mine + lane * kV * NC, av, t_agg);
+        }
+        Map acc[kV];
+#pragma unroll
+        for (int j = 0; j < kV; ++j) acc[j] = Map::identity();
+        int jt = ticket - stride;
+        bool done = false;
+        uint64_t t0 = 0;
+        unsigned spins = 0;
+        while (__any_sync(0xffffffffu, !done)) {
+            if (!done) {
+                const unsigned long long* pd = desc + (size_t)jt * TD::words;
+                float iv[kV * NS];
+                if (fetch_words(pd + TD::agg_words + lane * kV * NS, iv, t_incl)) {
+#pragma unroll
+                    for (int j = 0; j < kV; ++j) {
+                        float x[NS], y[NS];
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) x[q] = iv[j * NS + q];
+                        apply(acc[j], x, y);
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) carry[q][j] = y[q];
+                    }
+                    done = true;
+                } else {
+                    float av[kV * NC];
+                    if (fetch_words(pd + lane * kV * NC, av, t_agg)) {
+#pragma unroll
+                        for (int j = 0; j < kV; ++j) {
+                            Map e;
+#pragma unroll
+                            for (int i = 0; i < NC; ++i) e.set(i, av[j * NC + i]);
+                            acc[j] = compose(acc[j], e);
+                        }
+                        jt -= stride;
+                        spins = 0;
+                    } else {
+                        // predecessor not published yet: back off, bounded
+                        if ((++spins & 15u) == 0u) {
+                            if (error_raised(err)) {
+                                ok = false;
+                                done = true;
+                            } else {
+                                const uint64_t now = global_timer_ns();
+                                if (t0 == 0) {
+                                    t0 = now;
+                                } else if (now - t0 > wait_ns) {
+                                    raise_error(err, PARARNN_ERR_TIMEOUT);
+                                    ok = false;
+                                    done = true;
+                                }
+                            }
+                        }
+                        if (spins > 32) __nanosleep(64);
+                    }
+                }
+            }
+        }
+    }
+    if (ok) {
+        float iv[kV * NS];
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+            float x[NS], y[NS];
+#pragma unroll
+            for (int q = 0; q < NS; ++q) x[q] = carry[q][j];
+            apply(ta[j], x, y);
+#pragma unroll
+            for (int q = 0; q < NS; ++q) iv[j * NS + q] = y[q];
+        }
+        publish_words(mine + TD::agg_words + lane * kV * NS, iv, t_incl);
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+}  // namespace pararnn

@@ -1,0 +1,119 @@
+"""The C-ABI library on the CPU (no GPU needed): it loads, exports every entry
+point the header declares, sizes workspaces, and rejects bad arguments before
+queueing any GPU work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pararnn.h")
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from nonlinear_rnn_newton_b200 import build
+    build.build()
+    from nonlinear_rnn_newton_b200 import capi
+    return capi
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"PARARNN_API[^;(]*?\b(pararnn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ("pararnn_gru_solve", "pararnn_lstm_solve", "pararnn_gru_adjoint", "pararnn_lstm_adjoint",
+              "pararnn_gru_workspace_size", "pararnn_read_result", "pararnn_gru_sequential",
+              "pararnn_linear_scan", "pararnn_status_string", "pararnn_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(capi):
+    lib = ctypes.CDLL(capi.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+    # and the binding wraps every one of them
+    assert set(declared_symbols()) <= set(capi.SIGNATURES)
+
+
+def test_version_and_status_strings(capi):
+    assert re.match(r"^\d+\.\d+\.\d+$", capi.version())
+    assert capi.status_string(0) == "ok"
+    assert "timed out" in capi.status_string(-4)
+    assert capi.status_string(123) == "unknown status"
+
+
+def test_workspace_sizes(capi):
+    from nonlinear_rnn_newton_b200 import capi as c
+    g = c.pararnn_gru_workspace_size(8, 4096, 1024)
+    l = c.pararnn_lstm_workspace_size(8, 4096, 1024)
+    assert 0 < g < l
+    assert g % 256 == 0 and l % 256 == 0
+    assert c.pararnn_gru_workspace_size(8, 4096, 1020) == 0  # D not a multiple of 8
+    assert c.pararnn_gru_workspace_size(0, 4096, 1024) == 0
+    assert c.pararnn_gru_adjoint_workspace_size(4, 16384, 2048) > 0
+    assert c.pararnn_lstm_adjoint_workspace_size(4, 16384, 2048) > 0
+    assert c.pararnn_linear_scan_workspace_size(1, 65536, 2048) > 0
+    # monotone in every dimension
+    assert c.pararnn_gru_workspace_size(8, 8192, 1024) > g
+    assert c.pararnn_gru_workspace_size(16, 4096, 1024) > g
+
+
+def _solve(capi, u=16, a=16, h0=None, h=16, B=1, L=8, D=16, tol=1e-6, it=10, ws=256, wsb=1 << 30, dt=1):
+    lib = capi.lib
+    return lib.pararnn_gru_solve(u, dt, a, h0, h, B, L, D, tol, it, ws, wsb, None, None, None)
+
+
+def test_argument_checks_before_any_gpu_work(capi):
+    E = capi
+    assert _solve(capi, u=None) == E.ERR_INVALID_ARG
+    assert "u is NULL" in capi.last_error()
+    assert _solve(capi, a=None) == E.ERR_INVALID_ARG
+    assert _solve(capi, h=None) == E.ERR_INVALID_ARG
+    assert _solve(capi, u=8) == E.ERR_INVALID_ARG  # misaligned
+    assert "aligned" in capi.last_error()
+    assert _solve(capi, D=12) == E.ERR_UNSUPPORTED
+    assert _solve(capi, B=0) == E.ERR_INVALID_ARG
+    assert _solve(capi, L=-3) == E.ERR_INVALID_ARG
+    assert _solve(capi, tol=-1.0) == E.ERR_INVALID_ARG
+    assert _solve(capi, tol=float("inf")) == E.ERR_INVALID_ARG
+    assert _solve(capi, tol=float("nan")) == E.ERR_INVALID_ARG
+    assert _solve(capi, it=-1) == E.ERR_INVALID_ARG
+    assert _solve(capi, dt=7) == E.ERR_INVALID_ARG
+    assert _solve(capi, ws=None) == E.ERR_WORKSPACE
+    assert _solve(capi, ws=16) == E.ERR_WORKSPACE  # not 256-byte aligned
+    assert _solve(capi, wsb=100) == E.ERR_WORKSPACE
+    assert _solve(capi, B=1 << 20, L=1 << 20, D=1 << 10) == E.ERR_INVALID_ARG  # too large
+    lib = capi.lib
+    # LSTM, adjoints and baselines check too
+    assert lib.pararnn_lstm_solve(16, 1, 16, None, None, None, 16, 1, 8, 16, 1e-6, 10, 256, 1 << 30, None,
+                                  None, None) == E.ERR_INVALID_ARG
+    assert lib.pararnn_gru_adjoint(16, 1, 16, None, 16, None, 16, 16, None, 1, 8, 16, 256, 1 << 30,
+                                   None) == E.ERR_INVALID_ARG
+    assert lib.pararnn_lstm_adjoint(16, 1, 16, None, None, 16, 16, 16, None, 16, 16, None, None, 1, 8, 12,
+                                    256, 1 << 30, None) == E.ERR_UNSUPPORTED
+    assert lib.pararnn_gru_sequential(16, 1, None, None, 16, 1, 8, 16, None) == E.ERR_INVALID_ARG
+    assert lib.pararnn_linear_scan(16, 1, None, 16, 1, 8, 16, 256, 10, None) == E.ERR_WORKSPACE
+    assert lib.pararnn_selftest_wait_timeout(5, 10, 256, 16384, None) == E.ERR_INVALID_ARG
+
+
+def test_valid_arguments_without_gpu_report_cuda_error(capi):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _solve(capi) == capi.ERR_CUDA
+    assert capi.last_error()
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "capi_copy", os.path.join(ROOT, "nonlinear_rnn_newton_b200", "capi.py"))
+    mod = importlib.util.module_from_spec(spec)
+    monkeypatch.setattr(os.path, "exists", lambda p: False if p.endswith("libpararnn.so") else True)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)
