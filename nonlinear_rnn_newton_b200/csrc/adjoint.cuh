@@ -58,6 +58,7 @@ struct AdjointLayout {
     static constexpr size_t off_misc = off_carry + size_t(NS) * kDc * 4;
     static constexpr size_t smem_bytes = off_misc + 64;
     static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
+    static_assert(smem_bytes <= 232448, "shared memory");
 };
 
 template <class Cell, class UT, int T>

@@ -412,10 +412,38 @@ __device__ __forceinline__ void set_offset2(Aff2<2>& a, const float2* off)
     a.v1 = off[1];
 }
 
+// Jacobian pairs as plain arrays jm[entry][pair] (for shared-memory staging).
+template <int NJ>
+__device__ __forceinline__ void store_jacobian(const Jac2_1& a, float2 (&jm)[NJ][2], int jp) { jm[0][jp] = a.m; }
+
+template <int NJ>
+__device__ __forceinline__ void store_jacobian(const Jac2_2& a, float2 (&jm)[NJ][2], int jp)
+{
+    jm[0][jp] = a.m00;
+    jm[1][jp] = a.m01;
+    jm[2][jp] = a.m10;
+    jm[3][jp] = a.m11;
+}
+
+__device__ __forceinline__ void matrix_times2(const float2 (&jm)[1][2], int jp, const float2* x, float2* y)
+{
+    y[0] = mul2(jm[0][jp], x[0]);
+}
+
+__device__ __forceinline__ void matrix_times2(const float2 (&jm)[4][2], int jp, const float2* x, float2* y)
+{
+    y[0] = fma2(jm[0][jp], x[0], mul2(jm[1][jp], x[1]));
+    y[1] = fma2(jm[2][jp], x[0], mul2(jm[3][jp], x[1]));
+}
+
 // Packed diagonal GRU: f and J = df/dh for two channels.
+struct GruPacked2;
+struct LstmPacked2;
+
 struct GruPacked {
     using Map2 = Aff2<1>;
     using Jac2 = Jac2_1;
+    using Rows2 = GruPacked2;
     static constexpr int NJ = 1;  // Jacobian entries kept per channel pair
 
     __device__ __forceinline__ static void value(const float2* s, const float2* u, const float2* a, float2* f)
@@ -447,6 +475,7 @@ struct GruPacked {
 struct LstmPacked {
     using Map2 = Aff2<2>;
     using Jac2 = Jac2_2;
+    using Rows2 = LstmPacked2;
 
     __device__ __forceinline__ static void value(const float2* s, const float2* u, const float2* a, float2* out)
     {
@@ -478,6 +507,177 @@ struct LstmPacked {
         J.m01 = dcdh;
         J.m10 = mul2(ot, f);
         J.m11 = fma2(mul2(fma2(neg2(o), o, o), a[2]), t, mul2(ot, dcdh));
+    }
+};
+
+// ------------------------------------------- two timesteps, shared reciprocals
+// Rows of a sweep are independent evaluations, so two of them can share the
+// reciprocal of a product of denominators: with P = p_a p_b,
+// 1/p_a = p_b / P and 1/p_b = p_a / P.  Exponents are clamped from above at
+// kMaxT4 (four denominators) or kMaxT (two) so that P stays below 2^121; the
+// clamp changes s(x) only where s(x) < 2^-30.
+constexpr float kMaxT4 = 30.0f;
+
+__device__ __forceinline__ float2 clamp_t2_at(float2 t, float hi)
+{
+    return make_float2(min_keep_nan(t.x, hi), min_keep_nan(t.y, hi));
+}
+
+__device__ __forceinline__ float2 logistic_den2(float2 x, float hi)
+{
+    return add2(ex2_2(clamp_t2_at(mul2(bc2(-kLog2e), x), hi)), bc2(1.0f));
+}
+
+__device__ __forceinline__ float2 tanh_den2(float2 x, float hi)
+{
+    return add2(ex2_2(clamp_t2_at(mul2(bc2(2.0f * kLog2e), x), hi)), bc2(1.0f));
+}
+
+// 1/(da db) -> (1/da, 1/db) with one reciprocal per lane
+__device__ __forceinline__ void rcp_pair(float2 da, float2 db, float2& ia, float2& ib)
+{
+    const float2 inv = rcp_2(mul2(da, db));
+    ia = mul2(db, inv);
+    ib = mul2(da, inv);
+}
+
+// s(x_a), s(y_a), s(x_b), s(y_b) with one reciprocal per lane
+__device__ __forceinline__ void sigmoid4_2(float2 xa, float2 ya, float2 xb, float2 yb, float2& sxa, float2& sya,
+                                           float2& sxb, float2& syb)
+{
+    const float2 dxa = logistic_den2(xa, kMaxT4), dya = logistic_den2(ya, kMaxT4);
+    const float2 dxb = logistic_den2(xb, kMaxT4), dyb = logistic_den2(yb, kMaxT4);
+    const float2 pa = mul2(dxa, dya), pb = mul2(dxb, dyb);
+    float2 ia, ib;
+    rcp_pair(pa, pb, ia, ib);
+    sxa = mul2(dya, ia);
+    sya = mul2(dxa, ia);
+    sxb = mul2(dyb, ib);
+    syb = mul2(dxb, ib);
+}
+
+// s(x_a), tanh(y_a), s(x_b), tanh(y_b) with one reciprocal per lane
+__device__ __forceinline__ void sigmoid_tanh4_2(float2 xa, float2 ya, float2 xb, float2 yb, float2& sxa,
+                                                float2& tya, float2& sxb, float2& tyb)
+{
+    const float2 one = bc2(1.0f);
+    const float2 dxa = logistic_den2(xa, kMaxT4), dya = tanh_den2(ya, kMaxT4);
+    const float2 dxb = logistic_den2(xb, kMaxT4), dyb = tanh_den2(yb, kMaxT4);
+    const float2 pa = mul2(dxa, dya), pb = mul2(dxb, dyb);
+    float2 ia, ib;
+    rcp_pair(pa, pb, ia, ib);
+    sxa = mul2(dya, ia);
+    tya = fma2(mul2(bc2(-2.0f), dxa), ia, one);
+    sxb = mul2(dyb, ib);
+    tyb = fma2(mul2(bc2(-2.0f), dxb), ib, one);
+}
+
+// tanh(x_a), tanh(x_b) with one reciprocal per lane
+__device__ __forceinline__ void tanh2_2(float2 xa, float2 xb, float2& ta, float2& tb)
+{
+    const float2 one = bc2(1.0f);
+    float2 ia, ib;
+    rcp_pair(tanh_den2(xa, kMaxT), tanh_den2(xb, kMaxT), ia, ib);
+    ta = fma2(bc2(-2.0f), ia, one);
+    tb = fma2(bc2(-2.0f), ib, one);
+}
+
+// Two-row forms of the packed cells: rows a and b evaluated together.
+struct GruPacked2 {
+    // gates z, r, c at state h for rows a, b
+    __device__ __forceinline__ static void gates(float2 ha, const float2* ua, float2 hb, const float2* ub,
+                                                 const float2* a, float2& za, float2& ra, float2& ca, float2& zb,
+                                                 float2& rb, float2& cb)
+    {
+        sigmoid4_2(fma2(a[0], ha, ua[0]), fma2(a[1], ha, ua[1]), fma2(a[0], hb, ub[0]), fma2(a[1], hb, ub[1]), za,
+                   ra, zb, rb);
+        tanh2_2(fma2(a[2], mul2(ra, ha), ua[2]), fma2(a[2], mul2(rb, hb), ub[2]), ca, cb);
+    }
+
+    __device__ __forceinline__ static float2 jac(float2 h, float2 z, float2 r, float2 c, const float2* a)
+    {
+        const float2 one = bc2(1.0f);
+        const float2 cmh = fma2(h, bc2(-1.0f), c);
+        const float2 omz = fma2(z, bc2(-1.0f), one);
+        const float2 dr = fma2(mul2(h, a[1]), fma2(neg2(r), r, r), r);
+        const float2 dc = mul2(mul2(fma2(neg2(c), c, one), a[2]), dr);
+        return fma2(z, dc, fma2(mul2(mul2(z, omz), a[0]), cmh, omz));
+    }
+
+    __device__ __forceinline__ static void eval(const float2* sa, const float2* ua, const float2* sb,
+                                                const float2* ub, const float2* a, float2* fa, float2* fb,
+                                                Aff2<1>& Ja, Aff2<1>& Jb)
+    {
+        float2 za, ra, ca, zb, rb, cb;
+        gates(sa[0], ua, sb[0], ub, a, za, ra, ca, zb, rb, cb);
+        fa[0] = fma2(za, fma2(sa[0], bc2(-1.0f), ca), sa[0]);
+        fb[0] = fma2(zb, fma2(sb[0], bc2(-1.0f), cb), sb[0]);
+        Ja.m = jac(sa[0], za, ra, ca, a);
+        Jb.m = jac(sb[0], zb, rb, cb, a);
+    }
+
+    __device__ __forceinline__ static void value(const float2* sa, const float2* ua, const float2* sb,
+                                                 const float2* ub, const float2* a, float2* fa, float2* fb)
+    {
+        float2 za, ra, ca, zb, rb, cb;
+        gates(sa[0], ua, sb[0], ub, a, za, ra, ca, zb, rb, cb);
+        fa[0] = fma2(za, fma2(sa[0], bc2(-1.0f), ca), sa[0]);
+        fb[0] = fma2(zb, fma2(sb[0], bc2(-1.0f), cb), sb[0]);
+    }
+};
+
+struct LstmPacked2 {
+    __device__ __forceinline__ static void gates(float2 ha, const float2* ua, float2 hb, const float2* ub,
+                                                 const float2* a, float2 (&ga)[4], float2 (&gb)[4])
+    {
+        sigmoid4_2(fma2(a[0], ha, ua[0]), fma2(a[1], ha, ua[1]), fma2(a[0], hb, ub[0]), fma2(a[1], hb, ub[1]),
+                   ga[0], ga[1], gb[0], gb[1]);
+        sigmoid_tanh4_2(fma2(a[2], ha, ua[2]), fma2(a[3], ha, ua[3]), fma2(a[2], hb, ub[2]), fma2(a[3], hb, ub[3]),
+                        ga[2], ga[3], gb[2], gb[3]);
+    }
+
+    __device__ __forceinline__ static void jac(float2 c, const float2 (&g)[4], float2 t, const float2* a, Aff2<2>& J)
+    {
+        const float2 one = bc2(1.0f);
+        const float2 i = g[0], f = g[1], o = g[2], gg = g[3];
+        const float2 dcdh = fma2(mul2(c, a[1]), fma2(neg2(f), f, f),
+                                 fma2(mul2(gg, a[0]), fma2(neg2(i), i, i), mul2(mul2(i, fma2(neg2(gg), gg, one)), a[3])));
+        const float2 ot = mul2(o, fma2(neg2(t), t, one));
+        J.m00 = f;
+        J.m01 = dcdh;
+        J.m10 = mul2(ot, f);
+        J.m11 = fma2(mul2(fma2(neg2(o), o, o), a[2]), t, mul2(ot, dcdh));
+    }
+
+    __device__ __forceinline__ static void eval(const float2* sa, const float2* ua, const float2* sb,
+                                                const float2* ub, const float2* a, float2* fa, float2* fb,
+                                                Aff2<2>& Ja, Aff2<2>& Jb)
+    {
+        float2 ga[4], gb[4], ta, tb;
+        gates(sa[1], ua, sb[1], ub, a, ga, gb);
+        const float2 cna = fma2(ga[1], sa[0], mul2(ga[0], ga[3]));
+        const float2 cnb = fma2(gb[1], sb[0], mul2(gb[0], gb[3]));
+        tanh2_2(cna, cnb, ta, tb);
+        fa[0] = cna;
+        fa[1] = mul2(ga[2], ta);
+        fb[0] = cnb;
+        fb[1] = mul2(gb[2], tb);
+        jac(sa[0], ga, ta, a, Ja);
+        jac(sb[0], gb, tb, a, Jb);
+    }
+
+    __device__ __forceinline__ static void value(const float2* sa, const float2* ua, const float2* sb,
+                                                 const float2* ub, const float2* a, float2* fa, float2* fb)
+    {
+        float2 ga[4], gb[4], ta, tb;
+        gates(sa[1], ua, sb[1], ub, a, ga, gb);
+        const float2 cna = fma2(ga[1], sa[0], mul2(ga[0], ga[3]));
+        const float2 cnb = fma2(gb[1], sb[0], mul2(gb[0], gb[3]));
+        tanh2_2(cna, cnb, ta, tb);
+        fa[0] = cna;
+        fa[1] = mul2(ga[2], ta);
+        fb[0] = cnb;
+        fb[1] = mul2(gb[2], tb);
     }
 };
 

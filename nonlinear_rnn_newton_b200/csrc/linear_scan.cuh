@@ -35,6 +35,7 @@ struct LinScanLayout {
     static constexpr size_t off_misc = off_carry + size_t(kDc) * 4;
     static constexpr size_t smem_bytes = off_misc + 64;
     static constexpr int desc_words = TileDesc<Aff<1>, 1>::words;
+    static_assert(smem_bytes <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ Aff<1> linear_gru_map(float uz, float uc)

@@ -65,6 +65,75 @@ struct NewtonParams {
     unsigned long long wait_ns;
 };
 
+
+// Convergence decision after pass k, taken identically by every CTA from the
+// global residual maxima (see the stopping rule in pararnn.h).
+struct NewtonDecision {
+    int cont;    // run another pass
+    int zero;    // return the initial guess H^0 = 0
+    int iters, status;
+    float residual, residual0;
+};
+
+__device__ __forceinline__ NewtonDecision newton_decide(WsHeader* hdr, int k, int slot, bool bar_ok, float tol,
+                                                        int max_iters)
+{
+    NewtonDecision d{0, 0, k + 1, PARARNN_OK, 0.f, 0.f};
+    const unsigned post_bits = ld_acquire_gpu_u32(&hdr->res[slot]);
+    const unsigned pre_bits = ld_acquire_gpu_u32(&hdr->res0);
+    const float r0 = __uint_as_float(pre_bits);
+    const float rk = __uint_as_float(post_bits);
+    const int e = ld_relaxed_gpu(&hdr->error);
+    d.residual0 = r0;
+    d.residual = rk;
+    if (!bar_ok || e != 0) {
+        d.status = e != 0 ? e : PARARNN_ERR_TIMEOUT;
+        return d;
+    }
+    if (k == 0) {
+        if (pre_bits >= 0x7f800000u) {  // NaN or inf residual of the initial guess
+            d.status = PARARNN_ERR_NONFINITE;
+            d.iters = 0;
+            d.residual = r0;
+            d.zero = 1;
+            return d;
+        }
+        if (r0 <= tol || max_iters == 0) {
+            d.status = r0 <= tol ? PARARNN_OK : PARARNN_NOT_CONVERGED;
+            d.iters = 0;
+            d.residual = r0;
+            d.zero = 1;
+            return d;
+        }
+    }
+    if (post_bits >= 0x7f800000u) d.status = PARARNN_ERR_NONFINITE;
+    else if (rk <= tol) d.status = PARARNN_OK;
+    else if (k + 1 >= max_iters) d.status = PARARNN_NOT_CONVERGED;
+    else d.cont = 1;
+    return d;
+}
+
+__device__ __forceinline__ void newton_publish(WsHeader* hdr, const NewtonDecision& d, int k)
+{
+    hdr->result.status = d.status;
+    hdr->result.iters = d.iters;
+    hdr->result.residual = d.residual;
+    hdr->result.residual0 = d.residual0;
+    hdr->passes = k + 1;
+}
+
+// Converged (or stopped) at the initial guess: the states are H^0 = 0.
+template <int NS>
+__device__ __forceinline__ void newton_zero_states(const NewtonParams& p, int tid, int nthreads)
+{
+    const size_t n4 = size_t(p.B * p.L * p.D) / 4;
+    for (int q = 0; q < NS; ++q) {
+        float4* o = reinterpret_cast<float4*>(p.st[q]);
+        for (size_t i = size_t(blockIdx.x) * nthreads + tid; i < n4; i += size_t(gridDim.x) * nthreads)
+            o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
 template <class Cell, class UT, int T>
 struct NewtonLayout {
     static constexpr int G = Cell::G;
@@ -81,8 +150,10 @@ struct NewtonLayout {
     static constexpr size_t off_scan = 2 * stage_bytes;  // per-warp aggregates [NC][kWarps][kScanPad]
     static constexpr size_t off_carry = off_scan + size_t(NC) * kWarps * kScanPad * 4;  // [NS][kDc]
     static constexpr size_t off_misc = off_carry + size_t(NS) * kDc * 4;
-    static constexpr size_t smem_bytes = off_misc + 192;
+    // misc: 2 barriers per stage (32 B), 16 flags (64 B), 2*kWarps residual slots
+    static constexpr size_t smem_bytes = off_misc + ((96 + 8 * kWarps + 127) / 128) * 128;
     static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
+    static_assert(smem_bytes <= 232448, "shared memory");
     static_assert(u_bytes % 128 == 0 && stage_bytes % 128 == 0 && off_scan % 16 == 0, "alignment");
 };
 
@@ -448,68 +519,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
 
         const bool bar_ok = grid_barrier(&hdr->bar, unsigned(k), err, p.wait_ns, &s_int[2]);
 
-        // every CTA takes the same decision from the same global values
         if (tid == 0) {
-            int cont = 0, zero = 0, iters, status;
-            float resid;
-            const unsigned post_bits = ld_acquire_gpu_u32(&hdr->res[slot]);
-            const unsigned pre_bits = ld_acquire_gpu_u32(&hdr->res0);
-            const float r0 = __uint_as_float(pre_bits);
-            const float rk = __uint_as_float(post_bits);
-            const int e = ld_relaxed_gpu(err);
-            bool decided = false;
-            if (!bar_ok || e != 0) {
-                status = e != 0 ? e : PARARNN_ERR_TIMEOUT;
-                iters = k + 1;
-                resid = rk;
-                decided = true;
-            } else if (first) {
-                if (pre_bits >= 0x7f800000u) {
-                    status = PARARNN_ERR_NONFINITE;
-                    iters = 0;
-                    resid = r0;
-                    zero = 1;
-                    decided = true;
-                } else if (r0 <= p.tol || p.max_iters == 0) {
-                    status = r0 <= p.tol ? PARARNN_OK : PARARNN_NOT_CONVERGED;
-                    iters = 0;
-                    resid = r0;
-                    zero = 1;
-                    decided = true;
-                }
-            }
-            if (!decided) {
-                iters = k + 1;
-                resid = rk;
-                if (post_bits >= 0x7f800000u) status = PARARNN_ERR_NONFINITE;
-                else if (rk <= p.tol) status = PARARNN_OK;
-                else if (k + 1 >= p.max_iters) status = PARARNN_NOT_CONVERGED;
-                else {
-                    status = PARARNN_OK;
-                    cont = 1;
-                }
-            }
-            if (!cont && blockIdx.x == 0) {
-                hdr->result.status = status;
-                hdr->result.iters = iters;
-                hdr->result.residual = resid;
-                hdr->result.residual0 = r0;
-                hdr->passes = k + 1;
-            }
-            s_int[3] = cont;
-            s_int[4] = zero;
+            NewtonDecision d = newton_decide(hdr, k, slot, bar_ok, p.tol, p.max_iters);
+            if (!d.cont && blockIdx.x == 0) newton_publish(hdr, d, k);
+            s_int[3] = d.cont;
+            s_int[4] = d.zero;
         }
         __syncthreads();
         if (!s_int[3]) {
-            if (s_int[4]) {
-                // converged (or stopped) at the initial guess H^0 = 0
-                const size_t n4 = size_t(p.B * L * D) / 4;
-                for (int q = 0; q < NS; ++q) {
-                    float4* o = reinterpret_cast<float4*>(p.st[q]);
-                    for (size_t i = size_t(blockIdx.x) * kThreads + tid; i < n4; i += size_t(gridDim.x) * kThreads)
-                        o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
+            if (s_int[4]) newton_zero_states<NS>(p, tid, blockDim.x);
             return;
         }
         if (tid == 0) fence_proxy_async_global();  // other CTAs' state writes before our next TMA reads

@@ -1,0 +1,524 @@
+// Warp-specialised fused Newton solve (ParaGRU / ParaLSTM).
+//
+// Page: "ParaRNN: Apple destrava treino paralelo de RNNs não-lineares e escala
+// pra 7B parâmetros" -- "A sacada: método de Newton" (each iteration linearises
+// every step and solves the linear SSM delta_l = J_l delta_{l-1} - F_l with a
+// parallel scan), "Engenharia pra escalar" (diagonal / 2x2 Jacobians; Newton
+// iterations, system assembly and the parallel reduction fused in one kernel).
+//
+// The mathematics is that of newton.cuh (direct form of the Newton step
+// s^{k+1}_l = J_l s^{k+1}_{l-1} + o_l with o_l = f_l - J_l s^k_{l-1}; residual
+// of the updated states for the convergence test; grid barrier and a common
+// decision between iterations).  The work of a CTA is split by role so that
+// no CTA-wide barrier sits inside the tile loop:
+//   * CW compute warps, each owning two consecutive steps of a tile
+//     (tile = 2*CW steps x 128 channels).  For tile n a warp runs sweep 1
+//     (cell, Jacobian and offsets of its two steps, evaluated together so
+//     they share reciprocals; fold of its two maps), then sweep 2 of tile n-1
+//     (apply the carry, write the states, residual of the new states).  The
+//     Jacobians of the previous tile wait in registers, the offsets in
+//     shared memory.
+//   * one control warp takes tickets and issues the TMA loads into a
+//     three-stage ring, composes the compute warps' folds of tile n, runs the
+//     decoupled look-back against other CTAs and hands each compute warp the
+//     state entering its steps.
+// Hand-offs use mbarriers (full: loads landed; aggr: folds written; carry:
+// carries written; empty: stage released).  Every wait is bounded.
+#pragma once
+
+#include <climits>
+
+#include "newton.cuh"
+
+namespace pararnn {
+
+constexpr int kStages = 3;
+
+__device__ __forceinline__ float max_keep_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+template <class Cell, class UT, int CW>
+struct NewtonWsLayout {
+    static constexpr int G = Cell::G;
+    static constexpr int NS = Cell::NS;
+    static constexpr int NC = Cell::Map::kFloats;
+    static constexpr int Lc = 2 * CW;  // two steps per compute warp
+    static constexpr int kPad = kDc + 4;
+    static constexpr size_t a128(size_t x) { return (x + 127) & ~size_t(127); }
+    static constexpr size_t u_tx = size_t(Lc) * G * kDc * sizeof(UT);   // bytes one gate tile load delivers
+    static constexpr size_t s_tx = size_t(Lc) * kDc * 4;                 // bytes one state tile load delivers
+    static constexpr size_t u_bytes = a128(u_tx);
+    static constexpr size_t s_bytes = a128(s_tx);            // one state component
+    static constexpr size_t last_bytes = a128(size_t(NS) * CW * kDc * 4);    // offsets of each warp's 2nd step
+    static constexpr size_t agg_bytes = a128(size_t(NC) * CW * kPad * 4);    // warps' folds
+    static constexpr size_t carry_bytes = a128(size_t(NS) * CW * kDc * 4);   // state entering each warp
+    static constexpr size_t off_u = 0;
+    static constexpr size_t off_s = off_u + u_bytes;
+    static constexpr size_t off_last = off_s + NS * s_bytes;
+    static constexpr size_t off_agg = off_last + last_bytes;
+    static constexpr size_t off_carry = off_agg + agg_bytes;
+    static constexpr size_t stage_bytes = off_carry + carry_bytes;
+    static constexpr size_t off_misc = kStages * stage_bytes;
+    // misc: 4 barriers per stage, tickets, 8 flags, 2*(CW+1) residual slots
+    static constexpr size_t misc_bytes = a128(4 * kStages * 8 + kStages * 4 + 8 * 4 + 2 * (CW + 1) * 4);
+    static constexpr size_t smem_bytes = off_misc + misc_bytes;
+    static constexpr int threads = 32 * (CW + 1);
+    static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
+    static_assert(smem_bytes <= 232448, "shared memory");
+};
+
+template <class Cell, class UT, int CW>
+__global__ void __launch_bounds__(32 * (CW + 1), 1)
+    newton_solve_ws_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_s0,
+                           const __grid_constant__ CUtensorMap tm_s1, const NewtonParams p)
+{
+    using LY = NewtonWsLayout<Cell, UT, CW>;
+    using Map = typename Cell::Map;
+    using Packed = typename Cell::Packed;
+    using Rows2 = typename Packed::Rows2;
+    using Map2 = typename Packed::Map2;
+    using Jac2 = typename Packed::Jac2;
+    constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc, kPad = LY::kPad;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + LY::off_misc);  // [kStages]
+    uint64_t* bar_aggr = bar_full + kStages;
+    uint64_t* bar_carry = bar_aggr + kStages;
+    uint64_t* bar_empty = bar_carry + kStages;
+    int* s_tick = reinterpret_cast<int*>(bar_empty + kStages);  // [kStages]
+    int* s_int = s_tick + kStages;                              // misc flags
+    float* s_red = reinterpret_cast<float*>(s_int + 8);         // [2 * (CW + 1)]
+
+    const int tid = threadIdx.x;
+    const int w = tid >> 5;
+    const int lane = tid & 31;
+    const bool ctl = (w == CW);
+    WsHeader* hdr = p.hdr;
+    int* err = &hdr->error;
+    const long long D = p.D, L = p.L;
+    const int BS = int(p.B) * p.S;
+    const int Dpad = p.S * kDc;
+
+    if (tid == 0) {
+        prefetch_tensormap(&tm_u);
+        prefetch_tensormap(&tm_s0);
+        if (NS == 2) prefetch_tensormap(&tm_s1);
+    }
+
+    for (int k = 0;; ++k) {
+        const int slot = k % 3;
+        const bool first = (k == 0);
+        if (tid == 0) {
+            if (blockIdx.x == 0) {
+                // slot (k+1)%3 was last used two passes ago; every CTA is past it
+                hdr->tick[(k + 1) % 3] = 0u;
+                hdr->res[(k + 1) % 3] = 0u;
+            }
+            // fresh barriers every pass (no copy is in flight between passes)
+            for (int i = 0; i < kStages; ++i) {
+                if (k > 0) {
+                    mbar_inval(&bar_full[i]);
+                    mbar_inval(&bar_aggr[i]);
+                    mbar_inval(&bar_carry[i]);
+                    mbar_inval(&bar_empty[i]);
+                }
+                mbar_init(&bar_full[i], 1);
+                mbar_init(&bar_aggr[i], CW);
+                mbar_init(&bar_carry[i], 1);
+                mbar_init(&bar_empty[i], CW);
+            }
+            s_int[0] = 0;  // look-back failure seen by the control warp
+            fence_mbar_init();
+        }
+        __syncthreads();
+        float rpost = 0.f, rpre = 0.f;  // max |F|, NaN kept
+
+        if (ctl) {
+            // ------------------------------------------------ control warp
+            auto issue = [&](int t, int stage) {  // lane 0 only
+                if (error_raised(err) || s_int[0]) t = INT_MAX;
+                s_tick[stage] = t;
+                if (t < p.n_tiles) {
+                    const int c = t / BS, rem = t - (t / BS) * BS;
+                    const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
+                    unsigned char* st = smem + stage * LY::stage_bytes;
+                    fence_proxy_async_shared();
+                    const uint32_t bytes = uint32_t(LY::u_tx + (first ? 0 : NS * LY::s_tx));
+                    mbar_arrive_expect_tx(&bar_full[stage], bytes);
+                    tma_load_4d(st + LY::off_u, &tm_u, d0, 0, c * Lc, b, &bar_full[stage]);
+                    if (!first) {
+                        tma_load_3d(st + LY::off_s, &tm_s0, d0, c * Lc, b, &bar_full[stage]);
+                        if (NS == 2)
+                            tma_load_3d(st + LY::off_s + LY::s_bytes, &tm_s1, d0, c * Lc, b, &bar_full[stage]);
+                    }
+                } else {
+                    mbar_arrive(&bar_full[stage]);
+                }
+                return t;
+            };
+            int tk[kStages];
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < kStages; ++i) tk[i] = issue(int(atomicAdd(&hdr->tick[slot], 1u)), i);
+            }
+#pragma unroll
+            for (int i = 0; i < kStages; ++i) tk[i] = __shfl_sync(0xffffffffu, tk[i], 0);
+            for (int n = 0;; ++n) {
+                const int s = n % kStages;
+                const uint32_t par = uint32_t(n / kStages) & 1u;
+                int ticket = tk[0];
+                if (s == 1) ticket = tk[1];
+                if (s == 2) ticket = tk[2];
+                if (ticket >= p.n_tiles) break;
+                const int c = ticket / BS, rem = ticket - (ticket / BS) * BS;
+                const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
+                const int dch = d0 + lane * kV;
+                const bool chv = dch < D;
+                float init[NS][kV];
+#pragma unroll
+                for (int q = 0; q < NS; ++q) {
+                    F4 x{{0.f, 0.f, 0.f, 0.f}};
+                    if (c == 0 && chv && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+#pragma unroll
+                    for (int j = 0; j < kV; ++j) init[q][j] = x.v[j];
+                }
+                unsigned char* st = smem + s * LY::stage_bytes;
+                const float* agg = reinterpret_cast<const float*>(st + LY::off_agg);
+                float* car = reinterpret_cast<float*>(st + LY::off_carry);
+                bool ok = mbar_wait_bounded(&bar_aggr[s], par, err, p.wait_ns);
+                // tile aggregate = the warps' folds composed in step order
+                Map ta[kV];
+#pragma unroll
+                for (int j = 0; j < kV; ++j) ta[j] = Map::identity();
+                for (int seg = 0; seg < CW; ++seg) {
+                    Map m[kV];
+#pragma unroll
+                    for (int i = 0; i < NC; ++i) {
+                        F4 v = load4(agg + (i * CW + seg) * kPad + lane * kV);
+#pragma unroll
+                        for (int j = 0; j < kV; ++j) m[j].set(i, v.v[j]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < kV; ++j) ta[j] = compose(m[j], ta[j]);
+                }
+                float y[NS][kV];
+                ok = lookback<Map, NS>(ticket, BS, c > 0, k, ta, init, y, p.desc, lane, err, p.wait_ns) && ok;
+                // state entering each warp's steps
+                for (int seg = 0; seg < CW; ++seg) {
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) store4(car + (q * CW + seg) * kDc + lane * kV, y[q]);
+                    Map m[kV];
+#pragma unroll
+                    for (int i = 0; i < NC; ++i) {
+                        F4 v = load4(agg + (i * CW + seg) * kPad + lane * kV);
+#pragma unroll
+                        for (int j = 0; j < kV; ++j) m[j].set(i, v.v[j]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < kV; ++j) {
+                        float x[NS], z[NS];
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) x[q] = y[q][j];
+                        apply(m[j], x, z);
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) y[q][j] = z[q];
+                    }
+                }
+                if (!__all_sync(0xffffffffu, ok) && lane == 0) s_int[0] = 1;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_carry[s]);
+                // refill the stage released by the tile before this one
+                if (n >= 1) {
+                    const int sp = (n - 1) % kStages;
+                    int t = 0;
+                    if (lane == 0) {
+                        (void)mbar_wait_bounded(&bar_empty[sp], uint32_t((n - 1) / kStages) & 1u, err, p.wait_ns);
+                        t = issue(int(atomicAdd(&hdr->tick[slot], 1u)), sp);
+                    }
+                    t = __shfl_sync(0xffffffffu, t, 0);
+                    if (sp == 0) tk[0] = t;
+                    if (sp == 1) tk[1] = t;
+                    if (sp == 2) tk[2] = t;
+                }
+            }
+        } else {
+            // ------------------------------------------------ compute warps
+            const int ra = 2 * w, rb = 2 * w + 1;  // this warp's two steps in the tile
+            int prev_ticket = INT_MAX;
+            Jac2 Jp[2][2];  // Jacobians of the previous tile's two steps (per pair)
+            for (int n = 0;; ++n) {
+                const int s = n % kStages;
+                const uint32_t par = uint32_t(n / kStages) & 1u;
+                (void)mbar_wait_bounded(&bar_full[s], par, err, p.wait_ns);
+                const int ticket = s_tick[s];
+                const bool valid = ticket < p.n_tiles;
+                Jac2 Jn[2][2];
+                if (valid) {
+                    // ---- sweep 1 of tile n
+                    unsigned char* st = smem + s * LY::stage_bytes;
+                    const UT* su = reinterpret_cast<const UT*>(st + LY::off_u);
+                    float* ss = reinterpret_cast<float*>(st + LY::off_s);
+                    float* slast = reinterpret_cast<float*>(st + LY::off_last);
+                    float* sagg = reinterpret_cast<float*>(st + LY::off_agg);
+                    const int c = ticket / BS, rem = ticket - (ticket / BS) * BS;
+                    const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
+                    const int l0 = c * Lc;
+                    const int dch = d0 + lane * kV;
+                    const bool chv = dch < D;
+                    float2 wv[G][2];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        F4 x = chv ? load4(p.a + g * D + dch) : F4{{0.f, 0.f, 0.f, 0.f}};
+                        wv[g][0] = make_float2(x.v[0], x.v[1]);
+                        wv[g][1] = make_float2(x.v[2], x.v[3]);
+                    }
+                    // s^k before step a, s^k at steps a and b
+                    float2 sp[NS][2], ska[NS][2], skb[NS][2];
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) {
+                        F4 x{{0.f, 0.f, 0.f, 0.f}};
+                        if (w == 0) {
+                            if (chv) {
+                                if (c == 0) {
+                                    if (p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+                                } else if (!first) {
+                                    x = ldcg4(p.bnd + ((((size_t)(k & 1) * NS + q) * p.B + b) * p.n_chunks + (c - 1)) *
+                                                          Dpad + dch);
+                                }
+                            }
+                        } else if (!first) {
+                            x = load4(ss + (q * Lc + ra - 1) * kDc + lane * kV);
+                        }
+                        sp[q][0] = make_float2(x.v[0], x.v[1]);
+                        sp[q][1] = make_float2(x.v[2], x.v[3]);
+                        F4 xa{{0.f, 0.f, 0.f, 0.f}}, xb{{0.f, 0.f, 0.f, 0.f}};
+                        if (!first) {
+                            xa = load4(ss + (q * Lc + ra) * kDc + lane * kV);
+                            xb = load4(ss + (q * Lc + rb) * kDc + lane * kV);
+                        }
+                        ska[q][0] = make_float2(xa.v[0], xa.v[1]);
+                        ska[q][1] = make_float2(xa.v[2], xa.v[3]);
+                        skb[q][0] = make_float2(xb.v[0], xb.v[1]);
+                        skb[q][1] = make_float2(xb.v[2], xb.v[3]);
+                    }
+                    float2 ua[G][2], ub[G][2];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        F4 x = load4(su + (ra * G + g) * kDc + lane * kV);
+                        ua[g][0] = make_float2(x.v[0], x.v[1]);
+                        ua[g][1] = make_float2(x.v[2], x.v[3]);
+                        F4 z = load4(su + (rb * G + g) * kDc + lane * kV);
+                        ub[g][0] = make_float2(z.v[0], z.v[1]);
+                        ub[g][1] = make_float2(z.v[2], z.v[3]);
+                    }
+                    const bool va = (l0 + ra) < L && chv, vb = (l0 + rb) < L && chv;
+                    Map2 agg2[2];
+                    float2 offa[NS][2], offb[NS][2];
+#pragma unroll
+                    for (int jp = 0; jp < 2; ++jp) {
+                        float2 s_a[NS], s_b[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS], ja[NS], jb[NS];
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) {
+                            s_a[q] = sp[q][jp];
+                            s_b[q] = ska[q][jp];
+                        }
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            u_a[g] = ua[g][jp];
+                            u_b[g] = ub[g][jp];
+                            aa[g] = wv[g][jp];
+                        }
+                        Map2 ea, eb;
+                        Rows2::eval(s_a, u_a, s_b, u_b, aa, fa, fb, ea, eb);
+                        if (first) {
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) {
+                                const float2 da = add2(ska[q][jp], neg2(fa[q]));
+                                const float2 db = add2(skb[q][jp], neg2(fb[q]));
+                                if (va) rpre = max_keep_nan(rpre, max_keep_nan(fabsf(da.x), fabsf(da.y)));
+                                if (vb) rpre = max_keep_nan(rpre, max_keep_nan(fabsf(db.x), fabsf(db.y)));
+                            }
+                        }
+                        apply_matrix2(ea, s_a, ja);
+                        apply_matrix2(eb, s_b, jb);
+                        float2 oa[NS], ob[NS];
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) {
+                            oa[q] = fma2(ja[q], bc2(-1.0f), fa[q]);
+                            ob[q] = fma2(jb[q], bc2(-1.0f), fb[q]);
+                            offa[q][jp] = oa[q];
+                            offb[q][jp] = ob[q];
+                        }
+                        set_offset2(ea, oa);
+                        set_offset2(eb, ob);
+                        Jn[0][jp] = jacobian_of(ea);
+                        Jn[1][jp] = jacobian_of(eb);
+                        agg2[jp] = compose(eb, ea);
+                    }
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) {
+                        float va4[kV] = {offa[q][0].x, offa[q][0].y, offa[q][1].x, offa[q][1].y};
+                        float vb4[kV] = {offb[q][0].x, offb[q][0].y, offb[q][1].x, offb[q][1].y};
+                        store4(ss + (q * Lc + ra) * kDc + lane * kV, va4);  // step a's state is no longer read
+                        store4(slast + (q * CW + w) * kDc + lane * kV, vb4);  // step b's state is the next warp's input
+                    }
+                    {
+                        Map a1[kV] = {agg2[0].lane(0), agg2[0].lane(1), agg2[1].lane(0), agg2[1].lane(1)};
+#pragma unroll
+                        for (int i = 0; i < NC; ++i) {
+                            float v4[kV];
+#pragma unroll
+                            for (int j = 0; j < kV; ++j) v4[j] = a1[j].get(i);
+                            store4(sagg + (i * CW + w) * kPad + lane * kV, v4);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar_aggr[s]);
+                }
+                if (prev_ticket < p.n_tiles) {
+                    // ---- sweep 2 of tile n-1
+                    const int sp_ = (n - 1) % kStages;
+                    (void)mbar_wait_bounded(&bar_carry[sp_], uint32_t((n - 1) / kStages) & 1u, err, p.wait_ns);
+                    unsigned char* st = smem + sp_ * LY::stage_bytes;
+                    const UT* su = reinterpret_cast<const UT*>(st + LY::off_u);
+                    const float* ss = reinterpret_cast<const float*>(st + LY::off_s);
+                    const float* slast = reinterpret_cast<const float*>(st + LY::off_last);
+                    const float* car = reinterpret_cast<const float*>(st + LY::off_carry);
+                    const int t2 = prev_ticket;
+                    const int c = t2 / BS, rem = t2 - (t2 / BS) * BS;
+                    const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
+                    const int l0 = c * Lc;
+                    const int dch = d0 + lane * kV;
+                    const bool chv = dch < D && !s_int[0];
+                    float2 wv[G][2];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        F4 x = (dch < D) ? load4(p.a + g * D + dch) : F4{{0.f, 0.f, 0.f, 0.f}};
+                        wv[g][0] = make_float2(x.v[0], x.v[1]);
+                        wv[g][1] = make_float2(x.v[2], x.v[3]);
+                    }
+                    float2 y0[NS][2], offa[NS][2], offb[NS][2], ua[G][2], ub[G][2];
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) {
+                        F4 x = load4(car + (q * CW + w) * kDc + lane * kV);
+                        y0[q][0] = make_float2(x.v[0], x.v[1]);
+                        y0[q][1] = make_float2(x.v[2], x.v[3]);
+                        F4 xa = load4(ss + (q * Lc + ra) * kDc + lane * kV);
+                        F4 xb = load4(slast + (q * CW + w) * kDc + lane * kV);
+                        offa[q][0] = make_float2(xa.v[0], xa.v[1]);
+                        offa[q][1] = make_float2(xa.v[2], xa.v[3]);
+                        offb[q][0] = make_float2(xb.v[0], xb.v[1]);
+                        offb[q][1] = make_float2(xb.v[2], xb.v[3]);
+                    }
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        F4 x = load4(su + (ra * G + g) * kDc + lane * kV);
+                        ua[g][0] = make_float2(x.v[0], x.v[1]);
+                        ua[g][1] = make_float2(x.v[2], x.v[3]);
+                        F4 z = load4(su + (rb * G + g) * kDc + lane * kV);
+                        ub[g][0] = make_float2(z.v[0], z.v[1]);
+                        ub[g][1] = make_float2(z.v[2], z.v[3]);
+                    }
+                    const long long la = l0 + ra, lb = l0 + rb;
+                    const bool va = la < L && chv, vb = lb < L && chv;
+                    float2 ya[NS][2], yb[NS][2];
+#pragma unroll
+                    for (int jp = 0; jp < 2; ++jp) {
+                        float2 s0v[NS], sav[NS], sbv[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS], t0[NS], t1[NS];
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) s0v[q] = y0[q][jp];
+                        apply_matrix2(Jp[0][jp], s0v, t0);
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) sav[q] = add2(t0[q], offa[q][jp]);
+                        apply_matrix2(Jp[1][jp], sav, t1);
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) sbv[q] = add2(t1[q], offb[q][jp]);
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            u_a[g] = ua[g][jp];
+                            u_b[g] = ub[g][jp];
+                            aa[g] = wv[g][jp];
+                        }
+                        Rows2::value(s0v, u_a, sav, u_b, aa, fa, fb);
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) {
+                            const float2 da = add2(sav[q], neg2(fa[q]));
+                            const float2 db = add2(sbv[q], neg2(fb[q]));
+                            if (va) rpost = max_keep_nan(rpost, max_keep_nan(fabsf(da.x), fabsf(da.y)));
+                            if (vb) rpost = max_keep_nan(rpost, max_keep_nan(fabsf(db.x), fabsf(db.y)));
+                            ya[q][jp] = sav[q];
+                            yb[q][jp] = sbv[q];
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) {
+                        if (va)
+                            __stcg(reinterpret_cast<float4*>(p.st[q] + ((b * L + la) * D + dch)),
+                                   make_float4(ya[q][0].x, ya[q][0].y, ya[q][1].x, ya[q][1].y));
+                        if (vb)
+                            __stcg(reinterpret_cast<float4*>(p.st[q] + ((b * L + lb) * D + dch)),
+                                   make_float4(yb[q][0].x, yb[q][0].y, yb[q][1].x, yb[q][1].y));
+                    }
+                    if (w == CW - 1 && c + 1 < p.n_chunks && chv) {
+#pragma unroll
+                        for (int q = 0; q < NS; ++q)
+                            __stcg(reinterpret_cast<float4*>(
+                                       p.bnd + ((((size_t)((k + 1) & 1) * NS + q) * p.B + b) * p.n_chunks + c) *
+                                                   Dpad + dch),
+                                   make_float4(yb[q][0].x, yb[q][0].y, yb[q][1].x, yb[q][1].y));
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar_empty[sp_]);
+                }
+                if (!valid) break;
+                prev_ticket = ticket;
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int jp = 0; jp < 2; ++jp) Jp[r][jp] = Jn[r][jp];
+            }
+        }
+
+        // residual maxima of this CTA for this pass (max with NaN kept)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            rpost = max_keep_nan(rpost, __shfl_xor_sync(0xffffffffu, rpost, off));
+            rpre = max_keep_nan(rpre, __shfl_xor_sync(0xffffffffu, rpre, off));
+        }
+        if (lane == 0) {
+            s_red[w] = rpost;
+            s_red[CW + 1 + w] = rpre;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float a = 0.f, b2 = 0.f;
+            for (int i = 0; i <= CW; ++i) {
+                a = max_keep_nan(a, s_red[i]);
+                b2 = max_keep_nan(b2, s_red[CW + 1 + i]);
+            }
+            // non-negative floats (and NaN) order like their bit patterns
+            atomicMax(&hdr->res[slot], __float_as_uint(a) & 0x7fffffffu);
+            if (first) atomicMax(&hdr->res0, __float_as_uint(b2) & 0x7fffffffu);
+        }
+
+        const bool bar_ok = grid_barrier(&hdr->bar, unsigned(k), err, p.wait_ns, &s_int[1]);
+        if (tid == 0) {
+            NewtonDecision d = newton_decide(hdr, k, slot, bar_ok, p.tol, p.max_iters);
+            if (!d.cont && blockIdx.x == 0) newton_publish(hdr, d, k);
+            s_int[2] = d.cont;
+            s_int[3] = d.zero;
+        }
+        __syncthreads();
+        if (!s_int[2]) {
+            if (s_int[3]) newton_zero_states<NS>(p, tid, blockDim.x);
+            return;
+        }
+        if (tid == 0) fence_proxy_async_global();  // other CTAs' state writes before our next TMA reads
+    }
+}
+
+}  // namespace pararnn

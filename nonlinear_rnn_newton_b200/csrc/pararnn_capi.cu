@@ -18,6 +18,7 @@
 #include "device_common.cuh"
 #include "cells.cuh"
 #include "newton.cuh"
+#include "newton_ws.cuh"
 #include "sequential.cuh"
 #include "adjoint.cuh"
 #include "linear_scan.cuh"
@@ -51,6 +52,9 @@ pararnn_status fail(pararnn_status s, const char* fmt, ...)
         if (s_ != PARARNN_OK) return s_;          \
     } while (0)
 
+#ifndef PARARNN_WS
+#define PARARNN_WS 1
+#endif
 // Timesteps per warp in a tile (a tile has 8 warps).  Compile-time tuning
 // knobs; the workspace layout follows them.
 #ifndef PARARNN_GRU_ROWS
@@ -66,8 +70,28 @@ pararnn_status fail(pararnn_status s, const char* fmt, ...)
 #define PARARNN_LIN_ROWS 8
 #endif
 constexpr size_t kSelftestWorkspace = 16384;
-constexpr int kLcGru = kWarps * PARARNN_GRU_ROWS;    // GRU solve
-constexpr int kLcLstm = kWarps * PARARNN_LSTM_ROWS;  // LSTM solve
+#ifndef PARARNN_WS_GRU_WARPS
+#define PARARNN_WS_GRU_WARPS 16
+#endif
+#ifndef PARARNN_WS_LSTM_WARPS
+#define PARARNN_WS_LSTM_WARPS 8
+#endif
+#if PARARNN_WS
+// compute warps per CTA (two steps each); fp32 gates need twice the staging
+// space, so their tiles are half as long
+template <class UT> constexpr int gru_tile_arg() { return sizeof(UT) == 2 ? PARARNN_WS_GRU_WARPS : PARARNN_WS_GRU_WARPS / 2; }
+template <class UT> constexpr int lstm_tile_arg() { return sizeof(UT) == 2 ? PARARNN_WS_LSTM_WARPS : PARARNN_WS_LSTM_WARPS / 2; }
+template <class UT> constexpr int gru_lc() { return 2 * gru_tile_arg<UT>(); }
+template <class UT> constexpr int lstm_lc() { return 2 * lstm_tile_arg<UT>(); }
+#else
+template <class UT> constexpr int gru_tile_arg() { return PARARNN_GRU_ROWS; }
+template <class UT> constexpr int lstm_tile_arg() { return PARARNN_LSTM_ROWS; }
+template <class UT> constexpr int gru_lc() { return kWarps * PARARNN_GRU_ROWS; }
+template <class UT> constexpr int lstm_lc() { return kWarps * PARARNN_LSTM_ROWS; }
+#endif
+// workspace sizing uses the shortest tile (most tiles) of either input dtype
+constexpr int kLcGru = gru_lc<float>() < gru_lc<uint16_t>() ? gru_lc<float>() : gru_lc<uint16_t>();
+constexpr int kLcLstm = lstm_lc<float>() < lstm_lc<uint16_t>() ? lstm_lc<float>() : lstm_lc<uint16_t>();
 constexpr int kLcAdj = kWarps * PARARNN_ADJ_ROWS;    // adjoints
 constexpr int kLcLin = kWarps * PARARNN_LIN_ROWS;    // linear scan
 
@@ -209,14 +233,14 @@ pararnn_status device_info(int* sms)
 }
 
 template <class K>
-pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid)
+pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid, int threads = kThreads)
 {
     int sms = 0;
     TRY(device_info(&sms));
     CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   int(smem)));
     int occ = 0;
-    CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem));
+    CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem));
     if (occ < 1) return fail(PARARNN_ERR_CUDA, "kernel does not fit on an SM (smem %zu)", smem);
     *grid = std::max(1, std::min(n_tiles, occ * sms));
     return PARARNN_OK;
@@ -228,16 +252,27 @@ template <class Cell, class UT, int T>
 pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
                              float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream)
 {
-    using LY = NewtonLayout<Cell, UT, T>;
     constexpr int NS = Cell::NS;
-    const ScanLayout ly = scan_layout(s, LY::desc_words, solve_bnd_bytes(s, NS));
+    constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
+#if PARARNN_WS
+    using KL = NewtonWsLayout<Cell, UT, T>;  // T = compute warps (two steps each)
+    auto kern = newton_solve_ws_kernel<Cell, UT, T>;
+    constexpr int threads = KL::threads;
+#else
+    using KL = NewtonLayout<Cell, UT, T>;    // T = steps per warp
+    auto kern = newton_solve_kernel<Cell, UT, T>;
+    constexpr int threads = kThreads;
+#endif
+    // the TMA boxes must be exactly the kernel's tile
+    if (s.Lc != KL::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, KL::Lc);
+    const ScanLayout ly = scan_layout(s, desc_words, solve_bnd_bytes(s, NS));
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));  // header + descriptors
 
     CUtensorMap tu, t0, t1;
-    TRY(map_gates(&tu, u, dt, Cell::G, Cell::G, s, LY::Lc));
-    TRY(map_state(&t0, st[0], s, LY::Lc));
-    TRY(map_state(&t1, st[NS - 1], s, LY::Lc));
+    TRY(map_gates(&tu, u, dt, Cell::G, Cell::G, s, KL::Lc));
+    TRY(map_state(&t0, st[0], s, KL::Lc));
+    TRY(map_state(&t1, st[NS - 1], s, KL::Lc));
 
     NewtonParams p;
     p.a = a;
@@ -258,12 +293,11 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
     p.bnd = reinterpret_cast<float*>(wsb + ly.extra);
     p.wait_ns = kWaitLimitNs;
 
-    auto kern = newton_solve_kernel<Cell, UT, T>;
     int grid = 0;
-    TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid));
+    TRY(resident_grid(kern, KL::smem_bytes, s.n_tiles, &grid, threads));
     void* args[] = {(void*)&tu, (void*)&t0, (void*)&t1, (void*)&p};
-    CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(kThreads), args,
-                                         LY::smem_bytes, stream));
+    CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(threads), args,
+                                         KL::smem_bytes, stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return PARARNN_OK;
 }
@@ -277,8 +311,8 @@ size_t solve_ws_bytes(int cell, long long B, long long L, long long D)
     pararnn_status st = make_shape(B, L, D, cell == 0 ? kLcGru : kLcLstm, &s);
     memcpy(t_err, saved, sizeof(t_err));
     if (st != PARARNN_OK) return 0;
-    if (cell == 0) return scan_layout(s, NewtonLayout<GruCell, float, kLcGru / kWarps>::desc_words, solve_bnd_bytes(s, 1)).total;
-    return scan_layout(s, NewtonLayout<LstmCell, float, kLcLstm / kWarps>::desc_words, solve_bnd_bytes(s, 2)).total;
+    if (cell == 0) return scan_layout(s, TileDesc<Aff<1>, 1>::words, solve_bnd_bytes(s, 1)).total;
+    return scan_layout(s, TileDesc<Aff<2>, 2>::words, solve_bnd_bytes(s, 2)).total;
 }
 
 pararnn_status solve_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* c0, const float* h0,
@@ -303,15 +337,21 @@ pararnn_status solve_async(int cell, const void* u, pararnn_dtype dt, const floa
     if (cell == 0) {
         const float* s0[2] = {h0, nullptr};
         float* st[2] = {h, nullptr};
-        if (dt == PARARNN_BF16)
-            return launch_newton<GruCell, uint16_t, kLcGru / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
-        return launch_newton<GruCell, float, kLcGru / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+        if (dt == PARARNN_BF16) {
+            TRY(make_shape(B, L, D, gru_lc<uint16_t>(), &s));
+            return launch_newton<GruCell, uint16_t, gru_tile_arg<uint16_t>()>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+        }
+        TRY(make_shape(B, L, D, gru_lc<float>(), &s));
+        return launch_newton<GruCell, float, gru_tile_arg<float>()>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
     }
     const float* s0[2] = {c0, h0};
     float* st[2] = {c, h};
-    if (dt == PARARNN_BF16)
-        return launch_newton<LstmCell, uint16_t, kLcLstm / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
-    return launch_newton<LstmCell, float, kLcLstm / kWarps>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+    if (dt == PARARNN_BF16) {
+        TRY(make_shape(B, L, D, lstm_lc<uint16_t>(), &s));
+        return launch_newton<LstmCell, uint16_t, lstm_tile_arg<uint16_t>()>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+    }
+    TRY(make_shape(B, L, D, lstm_lc<float>(), &s));
+    return launch_newton<LstmCell, float, lstm_tile_arg<float>()>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
 }
 
 pararnn_status read_header(const void* ws, cudaStream_t stream, WsHeader* h)
@@ -361,6 +401,7 @@ pararnn_status launch_adjoint(const Shape& s, const void* u, pararnn_dtype dt, c
     CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));
 
     CUtensorMap tu, t0, t1, tg0, tg1;
+    if (s.Lc != LY::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, LY::Lc);
     TRY(map_gates(&tu, u, dt, G, G, s, LY::Lc));
     TRY(map_state(&t0, st[0], s, LY::Lc));
     TRY(map_state(&t1, st[NS - 1], s, LY::Lc));
@@ -467,6 +508,7 @@ pararnn_status launch_linear_scan(const Shape& s, const void* u, pararnn_dtype d
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));
     CUtensorMap tu1;
+    if (s.Lc != LY::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, LY::Lc);
     TRY(map_gates(&tu1, u, dt, 3, 1, s, LY::Lc));
     LinScanParams p;
     p.h0 = h0;
