@@ -32,6 +32,7 @@ from nonlinear_rnn_newton_b200 import workloads as W  # noqa: E402
 
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+METRIC = "Newton-solve tokens\u00b7channels/s and % of HBM roofline; iters to converge"
 
 
 def hbm_peak():
@@ -169,7 +170,7 @@ def time_baselines(w, xd, out, stream, reps=5):
         e1.record(stream)
         stream.synchronize()
         ms = e0.elapsed_time(e1) / reps
-        res[name] = {"ms": ms, "value": w.N / (ms * 1e-3), "unit": "tokens*channels/s",
+        res[name] = {"ms": ms, "value": w.N / (ms * 1e-3), "unit": "tokens\u00b7channels/s",
                      "gbs": nbytes / (ms * 1e-3) / 1e9}
     return res
 
@@ -205,13 +206,13 @@ def run_reference(args, w):
             vals.append(v)
     value = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": "Newton-solve tokens*channels/s", "value": value,
-        "unit": "tokens*channels/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": "tokens\u00b7channels/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * (w.L * w.D) / value, "higher_is_better": True, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name},
-        "cpu_baseline": {"value": value, "unit": "tokens*channels/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "tokens\u00b7channels/s", "cores": 1, "kind": "oracle",
                          "sample": desc},
-        "e2e": {"value": value, "unit": "tokens*channels/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": "tokens\u00b7channels/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "vs_baseline": None,
     }
     print(json.dumps(line), flush=True)
@@ -322,7 +323,7 @@ def main():
         e1.record(stream)
         stream.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
-        e2e = {"value": world * w.N / (ems * 1e-3), "unit": "tokens*channels/s", "ms_per_step": ems,
+        e2e = {"value": world * w.N / (ems * 1e-3), "unit": "tokens\u00b7channels/s", "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     baselines = None
@@ -332,11 +333,11 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, cores = cpu_oracle_sample(w, x, max_batches=1)
-        cpu = {"value": v, "unit": "tokens*channels/s", "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = {"value": v, "unit": "tokens\u00b7channels/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:
         line = {
-            "metric": "Newton-solve tokens*channels/s", "value": value, "unit": "tokens*channels/s",
+            "metric": METRIC, "value": value, "unit": "tokens\u00b7channels/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",

@@ -338,6 +338,12 @@ struct Aff2<1> {
     {
         return i == 0 ? Aff<1>{m.x, v.x} : Aff<1>{m.y, v.y};
     }
+    // entry i in the order of Aff<1>::get
+    __device__ __forceinline__ void set(int i, float2 x)
+    {
+        if (i == 0) m = x;
+        else v = x;
+    }
 };
 
 template <>
@@ -351,6 +357,18 @@ struct Aff2<2> {
     {
         return i == 0 ? Aff<2>{m00.x, m01.x, m10.x, m11.x, v0.x, v1.x}
                       : Aff<2>{m00.y, m01.y, m10.y, m11.y, v0.y, v1.y};
+    }
+    // entry i in the order of Aff<2>::get
+    __device__ __forceinline__ void set(int i, float2 x)
+    {
+        switch (i) {
+        case 0: m00 = x; break;
+        case 1: m01 = x; break;
+        case 2: m10 = x; break;
+        case 3: m11 = x; break;
+        case 4: v0 = x; break;
+        default: v1 = x; break;
+        }
     }
 };
 

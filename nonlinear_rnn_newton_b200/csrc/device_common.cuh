@@ -103,9 +103,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the warp is parked (issuing nothing) until
+// the phase completes or about `hint_ns` nanoseconds pass, so a waiting warp
+// does not take issue slots from the warps doing the arithmetic.
+__device__ __forceinline__ bool mbar_try_wait_parked(uint64_t* bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Longest single park of a bounded wait (ns); the time limit is checked
+// between parks.
+constexpr uint32_t kParkNs = 200000u;
+
 // ------------------------------------------------------------------------ TMA
 // Tiled bulk tensor loads into this CTA's shared memory, completing on an
 // mbarrier.  No multicast.
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(tm), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+        : "memory");
+}
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int c0, int c1, int c2,
                                             uint64_t* bar)
@@ -125,6 +154,21 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* tm, in
         " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
         "l"(tm), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
         : "memory");
+}
+
+// Tiled prefetch into L2 only (no shared memory, no completion tracking).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* tm, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tm), "r"(c0),
+                 "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* tm, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(tm), "r"(c0),
+                 "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm)
@@ -148,17 +192,13 @@ __device__ __forceinline__ bool error_raised(const int* err)
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
                                                   uint64_t limit_ns)
 {
-    uint64_t t0 = 0;
-    for (unsigned n = 0;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 15u) == 15u) {
-            uint64_t now = global_timer_ns();
-            if (t0 == 0) {
-                t0 = now;
-            } else if (now - t0 > limit_ns) {
-                raise_error(err, PARARNN_ERR_TIMEOUT);
-                return false;
-            }
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        if (mbar_try_wait_parked(bar, parity, kParkNs)) return true;
+        if (global_timer_ns() - t0 > limit_ns) {
+            raise_error(err, PARARNN_ERR_TIMEOUT);
+            return false;
         }
     }
 }

@@ -15,15 +15,21 @@
 //     (tile = 2*CW steps x 128 channels).  For tile n a warp runs sweep 1
 //     (cell, Jacobian and offsets of its two steps, evaluated together so
 //     they share reciprocals; fold of its two maps), then sweep 2 of tile n-1
-//     (apply the carry, write the states, residual of the new states).  The
-//     Jacobians of the previous tile wait in registers, the offsets in
-//     shared memory.
-//   * one control warp takes tickets and issues the TMA loads into a
-//     three-stage ring, composes the compute warps' folds of tile n, runs the
-//     decoupled look-back against other CTAs and hands each compute warp the
-//     state entering its steps.
+//     (state entering its steps = its prefix map applied to the tile's carry;
+//     the new states; residual of the new states).  The Jacobians of the
+//     previous tile wait in registers, the offsets in shared memory.
+//   * one control warp takes tickets (each worth a group of consecutive chunks
+//     of one sequence) and issues the TMA loads (gates, previous states, the
+//     slab's recurrence weights and the state entering the chunk from the
+//     last pass) into a four-stage ring; for tile n it starts the look-back's
+//     first read, turns the compute warps' folds into exclusive prefixes in
+//     place (their composition is the tile's aggregate), finishes the
+//     decoupled look-back against other CTAs -- or, inside a group, takes the
+//     inclusive value of the tile before -- and writes the tile's carry.
+// A tile's gates and states live in a ring stage from their load until its
+// sweep 2; the folds, offsets and carry live in one of two work buffers.
 // Hand-offs use mbarriers (full: loads landed; aggr: folds written; carry:
-// carries written; empty: stage released).  Every wait is bounded.
+// prefixes and carry written; empty: stage released).  Every wait is bounded.
 #pragma once
 
 #include <climits>
@@ -32,7 +38,24 @@
 
 namespace pararnn {
 
-constexpr int kStages = 3;
+#ifndef PARARNN_WS_STAGES
+#define PARARNN_WS_STAGES 4
+#endif
+constexpr int kStages = PARARNN_WS_STAGES;  // TMA ring
+constexpr int kWork = 2;    // per-tile work buffers (tiles n-1 and n are live)
+// A ticket hands out `group` consecutive chunks of one sequence; they run
+// back to back in one CTA, so only the first of them looks back across CTAs
+// (the others take their carry from the tile before, in registers).  This
+// shortens the chain of cross-CTA look-backs along a sequence, but the
+// chunks of a group then follow each other in time instead of running side
+// by side.  The 2x2-block cell, whose look-back steps are three times as
+// heavy, gains from groups of two; the diagonal cell does best without.
+#ifndef PARARNN_WS_GROUP_GRU
+#define PARARNN_WS_GROUP_GRU 1
+#endif
+#ifndef PARARNN_WS_GROUP_LSTM
+#define PARARNN_WS_GROUP_LSTM 2
+#endif
 
 __device__ __forceinline__ float max_keep_nan(float a, float b)
 {
@@ -47,24 +70,32 @@ struct NewtonWsLayout {
     static constexpr int NS = Cell::NS;
     static constexpr int NC = Cell::Map::kFloats;
     static constexpr int Lc = 2 * CW;  // two steps per compute warp
-    static constexpr int kPad = kDc + 4;
     static constexpr size_t a128(size_t x) { return (x + 127) & ~size_t(127); }
-    static constexpr size_t u_tx = size_t(Lc) * G * kDc * sizeof(UT);   // bytes one gate tile load delivers
-    static constexpr size_t s_tx = size_t(Lc) * kDc * 4;                 // bytes one state tile load delivers
-    static constexpr size_t u_bytes = a128(u_tx);
-    static constexpr size_t s_bytes = a128(s_tx);            // one state component
-    static constexpr size_t last_bytes = a128(size_t(NS) * CW * kDc * 4);    // offsets of each warp's 2nd step
-    static constexpr size_t agg_bytes = a128(size_t(NC) * CW * kPad * 4);    // warps' folds
-    static constexpr size_t carry_bytes = a128(size_t(NS) * CW * kDc * 4);   // state entering each warp
+    // bytes one load of each kind delivers
+    static constexpr size_t u_tx = size_t(Lc) * G * kDc * sizeof(UT);  // gate tile
+    static constexpr size_t s_tx = size_t(Lc) * kDc * 4;                // state tile, one component
+    static constexpr size_t a_tx = size_t(G) * kDc * 4;                 // recurrence weights of the slab
+    static constexpr size_t bnd_tx = size_t(kDc) * 4;                   // boundary row, one component
+    // ring stage: gates | states [NS] | weights | boundary [NS]
     static constexpr size_t off_u = 0;
-    static constexpr size_t off_s = off_u + u_bytes;
-    static constexpr size_t off_last = off_s + NS * s_bytes;
-    static constexpr size_t off_agg = off_last + last_bytes;
-    static constexpr size_t off_carry = off_agg + agg_bytes;
-    static constexpr size_t stage_bytes = off_carry + carry_bytes;
-    static constexpr size_t off_misc = kStages * stage_bytes;
-    // misc: 4 barriers per stage, tickets, 8 flags, 2*(CW+1) residual slots
-    static constexpr size_t misc_bytes = a128(4 * kStages * 8 + kStages * 4 + 8 * 4 + 2 * (CW + 1) * 4);
+    static constexpr size_t off_s = off_u + a128(u_tx);
+    static constexpr size_t s_bytes = a128(s_tx);
+    static constexpr size_t off_a = off_s + NS * s_bytes;
+    static constexpr size_t off_bnd = off_a + a128(a_tx);
+    static constexpr size_t stage_bytes = off_bnd + a128(NS * bnd_tx);
+    // work buffer: folds, then exclusive prefixes [NC][CW][kDc] | offsets of
+    // each warp's second step [NS][CW][kDc] | tile carry [NS][kDc]
+    static constexpr size_t off_agg = 0;
+    static constexpr size_t off_last = off_agg + a128(size_t(NC) * CW * kDc * 4);
+    static constexpr size_t off_carry = off_last + a128(size_t(NS) * CW * kDc * 4);
+    static constexpr size_t work_bytes = off_carry + a128(size_t(NS) * kDc * 4);
+    static constexpr size_t off_work = kStages * stage_bytes;
+    static constexpr size_t off_misc = off_work + kWork * work_bytes;
+    // misc: barriers (full, empty per stage; aggr, carry per work buffer), a
+    // job (ticket, chunk, batch row, first channel) per stage, 8 flags,
+    // 2*(CW+1) residual slots
+    static constexpr size_t misc_bytes =
+        a128((2 * kStages + 2 * kWork) * 8 + kStages * 16 + 8 * 4 + 2 * (CW + 1) * 4);
     static constexpr size_t smem_bytes = off_misc + misc_bytes;
     static constexpr int threads = 32 * (CW + 1);
     static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
@@ -74,7 +105,8 @@ struct NewtonWsLayout {
 template <class Cell, class UT, int CW>
 __global__ void __launch_bounds__(32 * (CW + 1), 1)
     newton_solve_ws_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_s0,
-                           const __grid_constant__ CUtensorMap tm_s1, const NewtonParams p)
+                           const __grid_constant__ CUtensorMap tm_s1, const __grid_constant__ CUtensorMap tm_a,
+                           const __grid_constant__ CUtensorMap tm_bnd, const NewtonParams p)
 {
     using LY = NewtonWsLayout<Cell, UT, CW>;
     using Map = typename Cell::Map;
@@ -82,16 +114,19 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
     using Rows2 = typename Packed::Rows2;
     using Map2 = typename Packed::Map2;
     using Jac2 = typename Packed::Jac2;
-    constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc, kPad = LY::kPad;
+    constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc;
+    constexpr int kGroup = NS == 1 ? PARARNN_WS_GROUP_GRU : PARARNN_WS_GROUP_LSTM;
 
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + LY::off_misc);  // [kStages]
-    uint64_t* bar_aggr = bar_full + kStages;
-    uint64_t* bar_carry = bar_aggr + kStages;
-    uint64_t* bar_empty = bar_carry + kStages;
-    int* s_tick = reinterpret_cast<int*>(bar_empty + kStages);  // [kStages]
-    int* s_int = s_tick + kStages;                              // misc flags
-    float* s_red = reinterpret_cast<float*>(s_int + 8);         // [2 * (CW + 1)]
+    uint64_t* bar_empty = bar_full + kStages;                                // [kStages]
+    uint64_t* bar_aggr = bar_empty + kStages;                                // [kWork]
+    uint64_t* bar_carry = bar_aggr + kWork;                                  // [kWork]
+    int4* s_job = reinterpret_cast<int4*>(bar_carry + kWork);                // [kStages]
+    int* s_int = reinterpret_cast<int*>(s_job + kStages);                    // misc flags
+    float* s_red = reinterpret_cast<float*>(s_int + 8);                      // [2 * (CW + 1)]
+    auto stage_at = [&](int i) { return smem + i * LY::stage_bytes; };
+    auto work_at = [&](int i) { return smem + LY::off_work + i * LY::work_bytes; };
 
     const int tid = threadIdx.x;
     const int w = tid >> 5;
@@ -107,6 +142,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
         prefetch_tensormap(&tm_u);
         prefetch_tensormap(&tm_s0);
         if (NS == 2) prefetch_tensormap(&tm_s1);
+        prefetch_tensormap(&tm_a);
+        prefetch_tensormap(&tm_bnd);
     }
 
     for (int k = 0;; ++k) {
@@ -122,14 +159,18 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
             for (int i = 0; i < kStages; ++i) {
                 if (k > 0) {
                     mbar_inval(&bar_full[i]);
-                    mbar_inval(&bar_aggr[i]);
-                    mbar_inval(&bar_carry[i]);
                     mbar_inval(&bar_empty[i]);
                 }
                 mbar_init(&bar_full[i], 1);
+                mbar_init(&bar_empty[i], CW);
+            }
+            for (int i = 0; i < kWork; ++i) {
+                if (k > 0) {
+                    mbar_inval(&bar_aggr[i]);
+                    mbar_inval(&bar_carry[i]);
+                }
                 mbar_init(&bar_aggr[i], CW);
                 mbar_init(&bar_carry[i], 1);
-                mbar_init(&bar_empty[i], CW);
             }
             s_int[0] = 0;  // look-back failure seen by the control warp
             fence_mbar_init();
@@ -141,138 +182,188 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
             // ------------------------------------------------ control warp
             auto issue = [&](int t, int stage) {  // lane 0 only
                 if (error_raised(err) || s_int[0]) t = INT_MAX;
-                s_tick[stage] = t;
                 if (t < p.n_tiles) {
                     const int c = t / BS, rem = t - (t / BS) * BS;
                     const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
-                    unsigned char* st = smem + stage * LY::stage_bytes;
+                    s_job[stage] = make_int4(t, c, b, d0);
+                    unsigned char* st = stage_at(stage);
                     fence_proxy_async_shared();
-                    const uint32_t bytes = uint32_t(LY::u_tx + (first ? 0 : NS * LY::s_tx));
+                    const bool with_bnd = !first && c > 0;  // state entering the chunk, from the last pass
+                    const uint32_t bytes = uint32_t(LY::u_tx + LY::a_tx + (first ? 0 : NS * LY::s_tx) +
+                                                    (with_bnd ? NS * LY::bnd_tx : 0));
                     mbar_arrive_expect_tx(&bar_full[stage], bytes);
                     tma_load_4d(st + LY::off_u, &tm_u, d0, 0, c * Lc, b, &bar_full[stage]);
+                    tma_load_2d(st + LY::off_a, &tm_a, d0, 0, &bar_full[stage]);
                     if (!first) {
                         tma_load_3d(st + LY::off_s, &tm_s0, d0, c * Lc, b, &bar_full[stage]);
                         if (NS == 2)
                             tma_load_3d(st + LY::off_s + LY::s_bytes, &tm_s1, d0, c * Lc, b, &bar_full[stage]);
                     }
+                    if (with_bnd) {
+#pragma unroll
+                        for (int q = 0; q < NS; ++q)
+                            tma_load_3d(st + LY::off_bnd + q * LY::bnd_tx, &tm_bnd, d0, c - 1,
+                                        ((k & 1) * NS + q) * int(p.B) + b, &bar_full[stage]);
+                    }
                 } else {
+                    s_job[stage] = make_int4(INT_MAX, 0, 0, 0);
                     mbar_arrive(&bar_full[stage]);
                 }
                 return t;
             };
+            // the next tile: the rest of the current group, then a new group
+            // ticket (lane 0 only; tickets count groups, tiles are numbered
+            // chunk * BS + sequence)
+            const int n_groups = ((p.n_chunks + kGroup - 1) / kGroup) * BS;
+            int g_c = 0, g_end = 0, g_q = 0;  // next chunk, end chunk and sequence of the group
+            auto next_tile = [&]() {
+                if (g_c >= g_end) {
+                    const int gt = int(atomicAdd(&hdr->tick[slot], 1u));
+                    if (gt >= n_groups) return INT_MAX;
+                    g_q = gt % BS;
+                    g_c = (gt / BS) * kGroup;
+                    g_end = min(g_c + kGroup, p.n_chunks);
+                }
+                return (g_c++) * BS + g_q;
+            };
+            // tickets of the tiles in the ring, by stage
             int tk[kStages];
             if (lane == 0) {
 #pragma unroll
-                for (int i = 0; i < kStages; ++i) tk[i] = issue(int(atomicAdd(&hdr->tick[slot], 1u)), i);
+                for (int i = 0; i < kStages; ++i) tk[i] = issue(next_tile(), i);
             }
 #pragma unroll
             for (int i = 0; i < kStages; ++i) tk[i] = __shfl_sync(0xffffffffu, tk[i], 0);
+            float y_inc[NS][kV];  // inclusive value of the last tile handled here
             for (int n = 0;; ++n) {
-                const int s = n % kStages;
-                const uint32_t par = uint32_t(n / kStages) & 1u;
+                const int s = n % kStages, wb = n % kWork;
                 int ticket = tk[0];
-                if (s == 1) ticket = tk[1];
-                if (s == 2) ticket = tk[2];
+#pragma unroll
+                for (int i = 1; i < kStages; ++i)
+                    if (s == i) ticket = tk[i];
                 if (ticket >= p.n_tiles) break;
                 const int c = ticket / BS, rem = ticket - (ticket / BS) * BS;
                 const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
                 const int dch = d0 + lane * kV;
-                const bool chv = dch < D;
+                // inside a group the tile before ran here: its inclusive value
+                // (y_inc) is this tile's carry
+                const bool local = (c % kGroup) != 0;
+                // first look-back read, in flight while the folds are composed
+                LookbackProbe<Map, NS> pr;
+                if (c > 0 && !local) lookback_probe(pr, ticket - BS, p.desc, lane);
                 float init[NS][kV];
 #pragma unroll
                 for (int q = 0; q < NS; ++q) {
                     F4 x{{0.f, 0.f, 0.f, 0.f}};
-                    if (c == 0 && chv && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+                    if (c == 0 && dch < D && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
 #pragma unroll
                     for (int j = 0; j < kV; ++j) init[q][j] = x.v[j];
                 }
-                unsigned char* st = smem + s * LY::stage_bytes;
-                const float* agg = reinterpret_cast<const float*>(st + LY::off_agg);
-                float* car = reinterpret_cast<float*>(st + LY::off_carry);
-                bool ok = mbar_wait_bounded(&bar_aggr[s], par, err, p.wait_ns);
-                // tile aggregate = the warps' folds composed in step order
-                Map ta[kV];
+                unsigned char* wk = work_at(wb);
+                float* agg = reinterpret_cast<float*>(wk + LY::off_agg);
+                float* car = reinterpret_cast<float*>(wk + LY::off_carry);
+                bool ok = mbar_wait_bounded(&bar_aggr[wb], uint32_t(n / kWork) & 1u, err, p.wait_ns);
+                // folds -> exclusive prefixes (in place); the last inclusive
+                // prefix is the tile's aggregate
+                Map run[kV];
 #pragma unroll
-                for (int j = 0; j < kV; ++j) ta[j] = Map::identity();
+                for (int j = 0; j < kV; ++j) run[j] = Map::identity();
                 for (int seg = 0; seg < CW; ++seg) {
                     Map m[kV];
 #pragma unroll
                     for (int i = 0; i < NC; ++i) {
-                        F4 v = load4(agg + (i * CW + seg) * kPad + lane * kV);
+                        float* row = agg + (i * CW + seg) * kDc + lane * kV;
+                        F4 v = load4(row);
+                        float v4[kV];
 #pragma unroll
-                        for (int j = 0; j < kV; ++j) m[j].set(i, v.v[j]);
+                        for (int j = 0; j < kV; ++j) {
+                            m[j].set(i, v.v[j]);
+                            v4[j] = run[j].get(i);
+                        }
+                        store4(row, v4);
                     }
 #pragma unroll
-                    for (int j = 0; j < kV; ++j) ta[j] = compose(m[j], ta[j]);
+                    for (int j = 0; j < kV; ++j) run[j] = compose(m[j], run[j]);
                 }
                 float y[NS][kV];
-                ok = lookback<Map, NS>(ticket, BS, c > 0, k, ta, init, y, p.desc, lane, err, p.wait_ns) && ok;
-                // state entering each warp's steps
-                for (int seg = 0; seg < CW; ++seg) {
+                if (local) {
 #pragma unroll
-                    for (int q = 0; q < NS; ++q) store4(car + (q * CW + seg) * kDc + lane * kV, y[q]);
-                    Map m[kV];
+                    for (int q = 0; q < NS; ++q)
 #pragma unroll
-                    for (int i = 0; i < NC; ++i) {
-                        F4 v = load4(agg + (i * CW + seg) * kPad + lane * kV);
+                        for (int j = 0; j < kV; ++j) y[q][j] = y_inc[q][j];
+                }
+                // the tile's inclusive value, kept for the next tile of the group
 #pragma unroll
-                        for (int j = 0; j < kV; ++j) m[j].set(i, v.v[j]);
-                    }
+                for (int j = 0; j < kV; ++j) {
+                    float x[NS], z[NS];
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) x[q] = y[q][j];
+                    apply(run[j], x, z);
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
+                }
+                if (local) {
+                    publish_inclusive<Map, NS>(p.desc, ticket, k, y_inc, lane);
+                } else {
+                    ok = lookback<Map, NS>(ticket, BS, c > 0, k, run, init, y, p.desc, lane, err, p.wait_ns, pr) && ok;
 #pragma unroll
                     for (int j = 0; j < kV; ++j) {
                         float x[NS], z[NS];
 #pragma unroll
                         for (int q = 0; q < NS; ++q) x[q] = y[q][j];
-                        apply(m[j], x, z);
+                        apply(run[j], x, z);
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) y[q][j] = z[q];
+                        for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
                     }
                 }
+#pragma unroll
+                for (int q = 0; q < NS; ++q) store4(car + q * kDc + lane * kV, y[q]);
                 if (!__all_sync(0xffffffffu, ok) && lane == 0) s_int[0] = 1;
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar_carry[s]);
+                if (lane == 0) mbar_arrive(&bar_carry[wb]);
                 // refill the stage released by the tile before this one
                 if (n >= 1) {
                     const int sp = (n - 1) % kStages;
                     int t = 0;
                     if (lane == 0) {
                         (void)mbar_wait_bounded(&bar_empty[sp], uint32_t((n - 1) / kStages) & 1u, err, p.wait_ns);
-                        t = issue(int(atomicAdd(&hdr->tick[slot], 1u)), sp);
+                        t = issue(next_tile(), sp);
                     }
                     t = __shfl_sync(0xffffffffu, t, 0);
-                    if (sp == 0) tk[0] = t;
-                    if (sp == 1) tk[1] = t;
-                    if (sp == 2) tk[2] = t;
+#pragma unroll
+                    for (int i = 0; i < kStages; ++i)
+                        if (sp == i) tk[i] = t;
                 }
             }
         } else {
             // ------------------------------------------------ compute warps
             const int ra = 2 * w, rb = 2 * w + 1;  // this warp's two steps in the tile
-            int prev_ticket = INT_MAX;
+            int4 prev = make_int4(INT_MAX, 0, 0, 0);  // job of the previous tile
             Jac2 Jp[2][2];  // Jacobians of the previous tile's two steps (per pair)
             for (int n = 0;; ++n) {
-                const int s = n % kStages;
-                const uint32_t par = uint32_t(n / kStages) & 1u;
-                (void)mbar_wait_bounded(&bar_full[s], par, err, p.wait_ns);
-                const int ticket = s_tick[s];
-                const bool valid = ticket < p.n_tiles;
+                const int s = n % kStages, wb = n % kWork;
+                (void)mbar_wait_bounded(&bar_full[s], uint32_t(n / kStages) & 1u, err, p.wait_ns);
+                const int4 job = s_job[s];
+                const bool valid = job.x < p.n_tiles;
                 Jac2 Jn[2][2];
                 if (valid) {
                     // ---- sweep 1 of tile n
-                    unsigned char* st = smem + s * LY::stage_bytes;
+                    unsigned char* st = stage_at(s);
+                    unsigned char* wk = work_at(wb);
                     const UT* su = reinterpret_cast<const UT*>(st + LY::off_u);
                     float* ss = reinterpret_cast<float*>(st + LY::off_s);
-                    float* slast = reinterpret_cast<float*>(st + LY::off_last);
-                    float* sagg = reinterpret_cast<float*>(st + LY::off_agg);
-                    const int c = ticket / BS, rem = ticket - (ticket / BS) * BS;
-                    const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
+                    const float* sa = reinterpret_cast<const float*>(st + LY::off_a);
+                    const float* sbnd = reinterpret_cast<const float*>(st + LY::off_bnd);
+                    float* slast = reinterpret_cast<float*>(wk + LY::off_last);
+                    float* sagg = reinterpret_cast<float*>(wk + LY::off_agg);
+                    const int c = job.y, b = job.z, d0 = job.w;
                     const int l0 = c * Lc;
                     const int dch = d0 + lane * kV;
                     const bool chv = dch < D;
                     float2 wv[G][2];
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        F4 x = chv ? load4(p.a + g * D + dch) : F4{{0.f, 0.f, 0.f, 0.f}};
+                        F4 x = load4(sa + g * kDc + lane * kV);  // zero beyond D (TMA fill)
                         wv[g][0] = make_float2(x.v[0], x.v[1]);
                         wv[g][1] = make_float2(x.v[2], x.v[3]);
                     }
@@ -282,13 +373,10 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     for (int q = 0; q < NS; ++q) {
                         F4 x{{0.f, 0.f, 0.f, 0.f}};
                         if (w == 0) {
-                            if (chv) {
-                                if (c == 0) {
-                                    if (p.s0[q]) x = load4(p.s0[q] + b * D + dch);
-                                } else if (!first) {
-                                    x = ldcg4(p.bnd + ((((size_t)(k & 1) * NS + q) * p.B + b) * p.n_chunks + (c - 1)) *
-                                                          Dpad + dch);
-                                }
+                            if (c == 0) {
+                                if (chv && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+                            } else if (!first) {
+                                x = load4(sbnd + q * kDc + lane * kV);
                             }
                         } else if (!first) {
                             x = load4(ss + (q * Lc + ra - 1) * kDc + lane * kV);
@@ -373,40 +461,65 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             float v4[kV];
 #pragma unroll
                             for (int j = 0; j < kV; ++j) v4[j] = a1[j].get(i);
-                            store4(sagg + (i * CW + w) * kPad + lane * kV, v4);
+                            store4(sagg + (i * CW + w) * kDc + lane * kV, v4);
                         }
                     }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar_aggr[s]);
+                    if (lane == 0) mbar_arrive(&bar_aggr[wb]);
                 }
-                if (prev_ticket < p.n_tiles) {
+                if (prev.x < p.n_tiles) {
                     // ---- sweep 2 of tile n-1
-                    const int sp_ = (n - 1) % kStages;
-                    (void)mbar_wait_bounded(&bar_carry[sp_], uint32_t((n - 1) / kStages) & 1u, err, p.wait_ns);
-                    unsigned char* st = smem + sp_ * LY::stage_bytes;
+                    const int sp_ = (n - 1) % kStages, wp = (n - 1) % kWork;
+                    (void)mbar_wait_bounded(&bar_carry[wp], uint32_t((n - 1) / kWork) & 1u, err, p.wait_ns);
+                    const unsigned char* st = stage_at(sp_);
+                    const unsigned char* wk = work_at(wp);
                     const UT* su = reinterpret_cast<const UT*>(st + LY::off_u);
                     const float* ss = reinterpret_cast<const float*>(st + LY::off_s);
-                    const float* slast = reinterpret_cast<const float*>(st + LY::off_last);
-                    const float* car = reinterpret_cast<const float*>(st + LY::off_carry);
-                    const int t2 = prev_ticket;
-                    const int c = t2 / BS, rem = t2 - (t2 / BS) * BS;
-                    const int b = rem / p.S, d0 = (rem - b * p.S) * kDc;
+                    const float* sa = reinterpret_cast<const float*>(st + LY::off_a);
+                    const float* slast = reinterpret_cast<const float*>(wk + LY::off_last);
+                    const float* spre = reinterpret_cast<const float*>(wk + LY::off_agg);
+                    const float* car = reinterpret_cast<const float*>(wk + LY::off_carry);
+                    const int c = prev.y, b = prev.z, d0 = prev.w;
                     const int l0 = c * Lc;
                     const int dch = d0 + lane * kV;
                     const bool chv = dch < D && !s_int[0];
                     float2 wv[G][2];
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        F4 x = (dch < D) ? load4(p.a + g * D + dch) : F4{{0.f, 0.f, 0.f, 0.f}};
+                        F4 x = load4(sa + g * kDc + lane * kV);
                         wv[g][0] = make_float2(x.v[0], x.v[1]);
                         wv[g][1] = make_float2(x.v[2], x.v[3]);
                     }
-                    float2 y0[NS][2], offa[NS][2], offb[NS][2], ua[G][2], ub[G][2];
+                    // state entering this warp's steps = its prefix map applied to the tile's carry
+                    float2 y0[NS][2];
+                    {
+                        Map2 pre[2];
+#pragma unroll
+                        for (int i = 0; i < NC; ++i) {
+                            F4 v = load4(spre + (i * CW + w) * kDc + lane * kV);
+                            pre[0].set(i, make_float2(v.v[0], v.v[1]));
+                            pre[1].set(i, make_float2(v.v[2], v.v[3]));
+                        }
+                        float2 ct[NS][2];
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) {
+                            F4 x = load4(car + q * kDc + lane * kV);
+                            ct[q][0] = make_float2(x.v[0], x.v[1]);
+                            ct[q][1] = make_float2(x.v[2], x.v[3]);
+                        }
+#pragma unroll
+                        for (int jp = 0; jp < 2; ++jp) {
+                            float2 x[NS], z[NS];
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) x[q] = ct[q][jp];
+                            apply2(pre[jp], x, z);
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) y0[q][jp] = z[q];
+                        }
+                    }
+                    float2 offa[NS][2], offb[NS][2], ua[G][2], ub[G][2];
 #pragma unroll
                     for (int q = 0; q < NS; ++q) {
-                        F4 x = load4(car + (q * CW + w) * kDc + lane * kV);
-                        y0[q][0] = make_float2(x.v[0], x.v[1]);
-                        y0[q][1] = make_float2(x.v[2], x.v[3]);
                         F4 xa = load4(ss + (q * Lc + ra) * kDc + lane * kV);
                         F4 xb = load4(slast + (q * CW + w) * kDc + lane * kV);
                         offa[q][0] = make_float2(xa.v[0], xa.v[1]);
@@ -475,7 +588,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     if (lane == 0) mbar_arrive(&bar_empty[sp_]);
                 }
                 if (!valid) break;
-                prev_ticket = ticket;
+                prev = job;
 #pragma unroll
                 for (int r = 0; r < 2; ++r)
 #pragma unroll

@@ -71,10 +71,10 @@ pararnn_status fail(pararnn_status s, const char* fmt, ...)
 #endif
 constexpr size_t kSelftestWorkspace = 16384;
 #ifndef PARARNN_WS_GRU_WARPS
-#define PARARNN_WS_GRU_WARPS 16
+#define PARARNN_WS_GRU_WARPS 15
 #endif
 #ifndef PARARNN_WS_LSTM_WARPS
-#define PARARNN_WS_LSTM_WARPS 8
+#define PARARNN_WS_LSTM_WARPS 7
 #endif
 #if PARARNN_WS
 // compute warps per CTA (two steps each); fp32 gates need twice the staging
@@ -221,6 +221,40 @@ pararnn_status map_state(CUtensorMap* m, const float* x, const Shape& s, int row
     return PARARNN_OK;
 }
 
+// Recurrence weights a [G][D] fp32: box = one slab of kDc channels, all gates.
+pararnn_status map_weights(CUtensorMap* m, const float* a, int G, const Shape& s)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {cuuint64_t(s.D), cuuint64_t(G)};
+    cuuint64_t strides[1] = {cuuint64_t(s.D) * 4};
+    cuuint32_t box[2] = {cuuint32_t(kDc), cuuint32_t(G)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled(weights) failed: %d", int(r));
+    return PARARNN_OK;
+}
+
+// Chunk boundary rows [2][NS][B][n_chunks][S*kDc] fp32, seen as 3-D
+// {D channels, n_chunks, 2*NS*B rows}: box = one slab of one row.
+pararnn_status map_bnd(CUtensorMap* m, const float* bnd, int NS, const Shape& s)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t row = cuuint64_t(s.S) * kDc * 4;
+    cuuint64_t dims[3] = {cuuint64_t(s.D), cuuint64_t(s.n_chunks), cuuint64_t(2) * NS * s.B};
+    cuuint64_t strides[2] = {row, row * cuuint64_t(s.n_chunks)};
+    cuuint32_t box[3] = {cuuint32_t(kDc), 1u, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(bnd), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled(boundary) failed: %d", int(r));
+    return PARARNN_OK;
+}
+
 pararnn_status device_info(int* sms)
 {
     int dev = 0;
@@ -295,7 +329,14 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
 
     int grid = 0;
     TRY(resident_grid(kern, KL::smem_bytes, s.n_tiles, &grid, threads));
+#if PARARNN_WS
+    CUtensorMap ta, tb;
+    TRY(map_weights(&ta, a, Cell::G, s));
+    TRY(map_bnd(&tb, p.bnd, NS, s));
+    void* args[] = {(void*)&tu, (void*)&t0, (void*)&t1, (void*)&ta, (void*)&tb, (void*)&p};
+#else
     void* args[] = {(void*)&tu, (void*)&t0, (void*)&t1, (void*)&p};
+#endif
     CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(threads), args,
                                          KL::smem_bytes, stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);

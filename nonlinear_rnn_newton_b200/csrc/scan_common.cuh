@@ -136,21 +136,45 @@ __device__ __forceinline__ void publish_words(unsigned long long* dst, const flo
     for (int i = 0; i < N; i += 2) st_words2(dst + i, tag_word(v[i], tag), tag_word(v[i + 1], tag));
 }
 
-// Load n (even) words; true if every tag equals `tag`.
+// Load n (even) words.
 template <int N>
-__device__ __forceinline__ bool fetch_words(const unsigned long long* src, float (&v)[N], unsigned tag)
+__device__ __forceinline__ void load_words(const unsigned long long* src, unsigned long long (&w)[N])
 {
     static_assert(N % 2 == 0, "pairs");
+#pragma unroll
+    for (int i = 0; i < N; i += 2) ld_words2(src + i, w[i], w[i + 1]);
+}
+
+// Values of n loaded words; true if every tag equals `tag`.
+template <int N>
+__device__ __forceinline__ bool unpack_words(const unsigned long long (&w)[N], float (&v)[N], unsigned tag)
+{
     bool ok = true;
 #pragma unroll
-    for (int i = 0; i < N; i += 2) {
-        unsigned long long a, b;
-        ld_words2(src + i, a, b);
-        ok = ok && unsigned(a >> 32) == tag && unsigned(b >> 32) == tag;
-        v[i] = __uint_as_float(unsigned(a));
-        v[i + 1] = __uint_as_float(unsigned(b));
+    for (int i = 0; i < N; ++i) {
+        ok = ok && unsigned(w[i] >> 32) == tag;
+        v[i] = __uint_as_float(unsigned(w[i]));
     }
     return ok;
+}
+
+// First look-back probe: the words of the predecessor tile (its inclusive
+// value and its aggregate), loaded early so that the round trip overlaps
+// whatever the caller does before calling lookback().
+template <class Map, int NS>
+struct LookbackProbe {
+    unsigned long long wi[kV * NS];
+    unsigned long long wa[kV * Map::kFloats];
+};
+
+template <class Map, int NS>
+__device__ __forceinline__ void lookback_probe(LookbackProbe<Map, NS>& pr, int pred_ticket,
+                                               const unsigned long long* desc, int lane)
+{
+    using TD = TileDesc<Map, NS>;
+    const unsigned long long* pd = desc + (size_t)pred_ticket * TD::words;
+    load_words(pd + TD::agg_words + lane * kV * NS, pr.wi);
+    load_words(pd + lane * kV * Map::kFloats, pr.wa);
 }
 
 // Decoupled look-back, run by one full warp; lane owns channels lane*kV..+kV-1.
@@ -159,15 +183,17 @@ __device__ __forceinline__ bool fetch_words(const unsigned long long* src, float
 //   epoch:     tags 2*epoch+1 (aggregate), 2*epoch+2 (inclusive)
 //   ta:        this tile's aggregate maps
 //   carry:     out: value entering this tile (the predecessors' inclusive)
+//   pr:        the first probe (lookback_probe of ticket - stride), if has_pred
 // Publishes the aggregate (if there is a predecessor) and, once the carry is
-// known, the inclusive value apply(ta, carry).  Each lane walks back on its
-// own; a wait that runs out of time raises PARARNN_ERR_TIMEOUT and returns
-// false.
+// known, the inclusive value apply(ta, carry).  Each step back reads the
+// predecessor's inclusive value and aggregate together (one round trip).
+// Each lane walks back on its own; a wait that runs out of time raises
+// PARARNN_ERR_TIMEOUT and returns false.
 template <class Map, int NS>
 __device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, int epoch, const Map (&ta)[kV],
                                          const float (&init)[NS][kV], float (&carry)[NS][kV],
                                          unsigned long long* desc, int lane, int* err,
-                                         unsigned long long wait_ns)
+                                         unsigned long long wait_ns, LookbackProbe<Map, NS>& pr)
 {
     using TD = TileDesc<Map, NS>;
     constexpr int NC = Map::kFloats;
@@ -196,9 +222,9 @@ __device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, 
         unsigned spins = 0;
         while (__any_sync(0xffffffffu, !done)) {
             if (!done) {
-                const unsigned long long* pd = desc + (size_t)jt * TD::words;
                 float iv[kV * NS];
-                if (fetch_words(pd + TD::agg_words + lane * kV * NS, iv, t_incl)) {
+                float av[kV * NC];
+                if (unpack_words(pr.wi, iv, t_incl)) {
 #pragma unroll
                     for (int j = 0; j < kV; ++j) {
                         float x[NS], y[NS];
@@ -209,37 +235,36 @@ __device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, 
                         for (int q = 0; q < NS; ++q) carry[q][j] = y[q];
                     }
                     done = true;
+                } else if (unpack_words(pr.wa, av, t_agg)) {
+#pragma unroll
+                    for (int j = 0; j < kV; ++j) {
+                        Map e;
+#pragma unroll
+                        for (int i = 0; i < NC; ++i) e.set(i, av[j * NC + i]);
+                        acc[j] = compose(acc[j], e);
+                    }
+                    jt -= stride;
+                    spins = 0;
+                    lookback_probe(pr, jt, desc, lane);
                 } else {
-                    float av[kV * NC];
-                    if (fetch_words(pd + lane * kV * NC, av, t_agg)) {
-#pragma unroll
-                        for (int j = 0; j < kV; ++j) {
-                            Map e;
-#pragma unroll
-                            for (int i = 0; i < NC; ++i) e.set(i, av[j * NC + i]);
-                            acc[j] = compose(acc[j], e);
-                        }
-                        jt -= stride;
-                        spins = 0;
-                    } else {
-                        // predecessor not published yet: back off, bounded
-                        if ((++spins & 15u) == 0u) {
-                            if (error_raised(err)) {
+                    // predecessor not published yet: back off, bounded
+                    if ((++spins & 15u) == 0u) {
+                        if (error_raised(err)) {
+                            ok = false;
+                            done = true;
+                        } else {
+                            const uint64_t now = global_timer_ns();
+                            if (t0 == 0) {
+                                t0 = now;
+                            } else if (now - t0 > wait_ns) {
+                                raise_error(err, PARARNN_ERR_TIMEOUT);
                                 ok = false;
                                 done = true;
-                            } else {
-                                const uint64_t now = global_timer_ns();
-                                if (t0 == 0) {
-                                    t0 = now;
-                                } else if (now - t0 > wait_ns) {
-                                    raise_error(err, PARARNN_ERR_TIMEOUT);
-                                    ok = false;
-                                    done = true;
-                                }
                             }
                         }
-                        if (spins > 32) __nanosleep(64);
                     }
+                    if (spins > 32) __nanosleep(64);
+                    if (!done) lookback_probe(pr, jt, desc, lane);
                 }
             }
         }
@@ -258,6 +283,33 @@ __device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, 
         publish_words(mine + TD::agg_words + lane * kV * NS, iv, t_incl);
     }
     return __all_sync(0xffffffffu, ok);
+}
+
+// Publish a tile's inclusive value when its carry is known without a
+// look-back (the tile before ran in the same CTA).
+template <class Map, int NS>
+__device__ __forceinline__ void publish_inclusive(unsigned long long* desc, int ticket, int epoch,
+                                                  const float (&incl)[NS][kV], int lane)
+{
+    using TD = TileDesc<Map, NS>;
+    float iv[kV * NS];
+#pragma unroll
+    for (int j = 0; j < kV; ++j)
+#pragma unroll
+        for (int q = 0; q < NS; ++q) iv[j * NS + q] = incl[q][j];
+    publish_words(desc + (size_t)ticket * TD::words + TD::agg_words + lane * kV * NS, iv, 2u * epoch + 2u);
+}
+
+// Look-back without an early probe.
+template <class Map, int NS>
+__device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, int epoch, const Map (&ta)[kV],
+                                         const float (&init)[NS][kV], float (&carry)[NS][kV],
+                                         unsigned long long* desc, int lane, int* err,
+                                         unsigned long long wait_ns)
+{
+    LookbackProbe<Map, NS> pr;
+    if (has_pred) lookback_probe(pr, ticket - stride, desc, lane);
+    return lookback<Map, NS>(ticket, stride, has_pred, epoch, ta, init, carry, desc, lane, err, wait_ns, pr);
 }
 
 }  // namespace pararnn
