@@ -155,6 +155,35 @@ PARARNN_API pararnn_status pararnn_lstm_solve_async(const void* u, pararnn_dtype
 PARARNN_API pararnn_status pararnn_read_result(const void* workspace, pararnn_stream_t stream,
                                    pararnn_result* result);
 
+/* ------------------------------------------------- fixed-scratch solve */
+
+/* ParaGRU Newton solve without a caller workspace.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory at the point of the call -- a plain C host program or a
+ * plugin that owns no device allocator, or a latency-critical loop that must
+ * not call cudaMalloc (which can synchronise the device) -- and so cannot
+ * provide the workspace pararnn_gru_solve needs.
+ *
+ * Its scratch is one fixed array of pararnn_gru_solve_noalloc_max_scratch()
+ * bytes (16 MiB) per device, part of the library's module image; the call
+ * allocates nothing (no cudaMalloc, no cudaFree, no other allocator).
+ * Shapes whose pararnn_gru_workspace_size exceeds that return
+ * PARARNN_ERR_WORKSPACE, before any device call, with the sizes in
+ * pararnn_last_error().  The first call on a device looks up the scratch's
+ * device address (cudaGetSymbolAddress, with that device current) and caches
+ * it: make that first call before capturing `stream` into a graph.  The
+ * scratch is shared by every call on the device, so calls that overlap in
+ * time (other threads, or other streams not yet finished) race and must be
+ * serialised by the caller.  Arguments, outputs and return values are those
+ * of pararnn_gru_solve; synchronous. */
+PARARNN_API pararnn_status pararnn_gru_solve_noalloc(const void* u, pararnn_dtype u_dtype, const float* a,
+                                         const float* h0, float* h, int64_t B, int64_t L, int64_t D,
+                                         float tol, int max_iters, pararnn_stream_t stream,
+                                         int* iters_out, float* residual_out);
+
+/* Bytes of the fixed scratch behind pararnn_gru_solve_noalloc. */
+PARARNN_API size_t pararnn_gru_solve_noalloc_max_scratch(void);
+
 /* -------------------------------------------------------------- adjoints */
 
 /* Gradients of a loss through the converged ParaGRU states.  The pages do

@@ -17,6 +17,8 @@ __all__ = [
     "pararnn_gru_sequential",
     "pararnn_gru_solve",
     "pararnn_gru_solve_async",
+    "pararnn_gru_solve_noalloc",
+    "pararnn_gru_solve_noalloc_max_scratch",
     "pararnn_gru_workspace_size",
     "pararnn_linear_scan",
     "pararnn_linear_scan_workspace_size",

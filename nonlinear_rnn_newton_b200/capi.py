@@ -55,6 +55,10 @@ SIGNATURES = {
                                 ctypes.POINTER(ctypes.c_float)]),
     "pararnn_gru_solve_async": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float,
                                       ctypes.c_int, _vp, ctypes.c_size_t, _vp]),
+    "pararnn_gru_solve_noalloc": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float,
+                                        ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_int),
+                                        ctypes.POINTER(ctypes.c_float)]),
+    "pararnn_gru_solve_noalloc_max_scratch": (ctypes.c_size_t, []),
     "pararnn_lstm_solve": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float,
                                  ctypes.c_int, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_int),
                                  ctypes.POINTER(ctypes.c_float)]),
@@ -216,6 +220,25 @@ def pararnn_gru_solve(u, a, h0=None, tol=1e-6, max_iters=10, h=None, workspace=N
         out.copy_(dh)
         dh = out
     return dh, it.value, res.value, st
+
+
+def pararnn_gru_solve_noalloc(u, a, h0, h, tol=1e-6, max_iters=10, stream=None):
+    """ParaGRU Newton solve on the library's fixed device scratch (no
+    workspace; device tensors only, h is the output).  Returns
+    (iters, residual, status)."""
+    B, L, G, D = u.shape
+    it = ctypes.c_int(0)
+    res = ctypes.c_float(0.0)
+    with torch.cuda.device(u.device):  # the scratch used is the current device's
+        st = lib.pararnn_gru_solve_noalloc(_ptr(u), _dtype_code(u), _ptr(a), _ptr(h0), _ptr(h), B, L, D,
+                                           float(tol), int(max_iters), _stream(u.device, stream),
+                                           ctypes.byref(it), ctypes.byref(res))
+    _check(st)
+    return it.value, res.value, st
+
+
+def pararnn_gru_solve_noalloc_max_scratch():
+    return lib.pararnn_gru_solve_noalloc_max_scratch()
 
 
 def pararnn_gru_solve_async(u, a, h0, h, workspace, tol=1e-6, max_iters=10, stream=None):

@@ -619,6 +619,37 @@ pararnn_status selftest_wait_timeout(int which, long long limit_ns, void* ws, si
     return PARARNN_OK;
 }
 
+// ------------------------------------------------ fixed scratch (no-alloc)
+//
+// Scratch of pararnn_gru_solve_noalloc: one array per device, part of this
+// library's module image, so using it needs no allocation call at all.  Its
+// address is looked up once per device (cudaGetSymbolAddress, with that
+// device current) and cached.  Calls that overlap in time on one device
+// share it and race.
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+constexpr int kNoAllocMaxDevices = 64;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+pararnn_status noalloc_scratch(void** out)
+{
+    int dev = -1;
+    CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(PARARNN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || !ptr)
+            return fail(PARARNN_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev, cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return PARARNN_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -643,6 +674,27 @@ pararnn_status pararnn_gru_solve(const void* u, pararnn_dtype u_dtype, const flo
     TRY(pararnn_gru_solve_async(u, u_dtype, a, h0, h, B, L, D, tol, max_iters, workspace, workspace_bytes, stream));
     return finish_sync(workspace, reinterpret_cast<cudaStream_t>(stream), iters_out, residual_out);
 }
+
+pararnn_status pararnn_gru_solve_noalloc(const void* u, pararnn_dtype u_dtype, const float* a, const float* h0,
+                                         float* h, int64_t B, int64_t L, int64_t D, float tol, int max_iters,
+                                         pararnn_stream_t stream, int* iters_out, float* residual_out)
+{
+    t_err[0] = '\0';
+    const size_t need = pararnn_gru_workspace_size(B, L, D);
+    if (need > kNoAllocScratchBytes)
+        return fail(PARARNN_ERR_WORKSPACE,
+                    "B=%lld L=%lld D=%lld needs %zu bytes of scratch; the fixed scratch holds %zu "
+                    "(use pararnn_gru_solve with a caller workspace)",
+                    (long long)B, (long long)L, (long long)D, need, kNoAllocScratchBytes);
+    void* ws = nullptr;
+    TRY(noalloc_scratch(&ws));
+    // the solve itself zeroes the scratch's header and tile descriptors on
+    // the stream before its kernel runs (as it does for any workspace)
+    return pararnn_gru_solve(u, u_dtype, a, h0, h, B, L, D, tol, max_iters, ws, kNoAllocScratchBytes, stream,
+                             iters_out, residual_out);
+}
+
+size_t pararnn_gru_solve_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
 
 pararnn_status pararnn_lstm_solve_async(const void* u, pararnn_dtype u_dtype, const float* a, const float* c0,
                                         const float* h0, float* c, float* h, int64_t B, int64_t L, int64_t D,
