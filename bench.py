@@ -1,22 +1,26 @@
 """Benchmark of the ParaRNN Newton solve on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-cpu-baseline]
+                    [--workload NAME] [--no-cpu-baseline] [--sweep]
 
-A step is one full Newton solve (every iteration until convergence) of the
-workload, through the C ABI (pararnn_*_solve_async), with inputs resident in
-HBM.  Default workload: ParaGRU, bf16 gate pre-activations / fp32 state,
-B=8, L=4096, D=1024 (u ~ N(0,1), a ~ U(-0.5,0.5), h0 ~ N(0,0.1), seed 0).
-Metric: tokens*channels per second = B*L*D / solve time.  Under torchrun
-every rank solves its own independent problem (seed + rank; no collective on
-the data path) and the time is the max over ranks.
+A step is one pass of the whole hot path over the workload through the C ABI:
+one full Newton solve (every iteration until convergence, the convergence
+test included) -- followed, for the training workload, by the reverse-time
+adjoint -- with inputs resident in HBM.  Default workload: ParaGRU, bf16 gate
+pre-activations / fp32 state, B=8, L=4096, D=1024 (u ~ N(0,1),
+a ~ U(-0.5,0.5), h0 ~ N(0,0.1), seed = rank).  Metric: tokens*channels per
+second = B*L*D / step time.  Under torchrun every rank solves its own
+independent problem (no collective on the data path) and the time is the max
+over ranks.
 
-Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle
-instead (the reference arm; rank 0 only).
+Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead (the reference arm; rank 0 only).
 """
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -31,27 +35,64 @@ import torch  # noqa: E402
 from nonlinear_rnn_newton_b200 import workloads as W  # noqa: E402
 
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+PROFILES = os.path.join(ROOT, "profiles")
+CSRC = os.path.join(ROOT, "nonlinear_rnn_newton_b200", "csrc")
 FALLBACK_HBM_GBS = 6650.0
-METRIC = "Newton-solve tokens\u00b7channels/s and % of HBM roofline; iters to converge"
+METRIC = "Newton-solve tokens·channels/s and % of HBM roofline; iters to converge"
+UNIT = "tokens·channels/s"
 
 
 def hbm_peak():
     try:
         with open(PEAKS_PATH) as f:
-            return float(json.load(f)["hbm_gbs"]), "measured"
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes(w: W.Workload, iters: int) -> int:
-    """Bytes a Newton solve must move: every pass reads the gates and writes the
-    states; every pass after the first (initial guess 0) also reads the states."""
+def solve_bytes(w: W.Workload, iters: int) -> int:
+    """Bytes a Newton solve must move: every pass reads the gates and writes
+    the states; every pass after the first (initial guess 0) also reads the
+    states.  Weights and workspace are < 0.1% and not counted."""
     es = 2 if w.u_dtype == "bf16" else 4
     ns = 1 if w.cell == "gru" else 2
-    per_first = w.G * es + ns * 4
-    per_next = w.G * es + 2 * ns * 4
-    passes = max(iters, 1)
-    return w.N * (per_first + (passes - 1) * per_next)
+    first = w.G * es + ns * 4
+    later = w.G * es + 2 * ns * 4
+    return w.N * (first + (max(iters, 1) - 1) * later)
+
+
+def adjoint_bytes(w: W.Workload) -> int:
+    """The adjoint reads gates, forward states (and the state before each
+    step, which is the previous row of the same arrays) and the upstream
+    gradient, and writes fp32 gate gradients."""
+    es = 2 if w.u_dtype == "bf16" else 4
+    ns = 1 if w.cell == "gru" else 2
+    return w.N * (w.G * es + ns * 4 + 4 + w.G * 4)
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when there is none or the kernel sources changed since
+    the counters were taken."""
+    path = os.path.join(PROFILES, f"{kernel}__{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
+    m_s = re.search(r"^source_digest:\s*([0-9a-f]+)", text, re.M)
+    if not m_t or not m_s or m_s.group(1) != source_digest():
+        return None
+    return int(m_t.group(1))
 
 
 class ClockSampler:
@@ -113,7 +154,7 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup(n_gpus):
+def dist_setup():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -126,13 +167,22 @@ def dist_setup(n_gpus):
     return rank, world, local
 
 
-def max_over_ranks(value, world):
+def max_over_ranks(value, world, device="cuda"):
+    """Max of a per-rank number over all ranks (every rank gets it); `device`
+    is where the backend's tensors live (cuda for nccl, cpu for gloo)."""
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(n_per_rank, world, ms_per_step):
+    """Whole-job throughput: every rank runs its own problem of n_per_rank
+    token*channels per step (weak scaling); the step time is the slowest
+    rank's."""
+    return world * n_per_rank / (ms_per_step * 1e-3)
 
 
 def barrier(world):
@@ -141,26 +191,76 @@ def barrier(world):
         dist.barrier()
 
 
-def solve_fn(w, xd, out, ws, stream):
-    import nonlinear_rnn_newton_b200 as P
-    if w.cell == "gru":
-        return lambda: P.pararnn_gru_solve_async(xd.u, xd.a, xd.h0, out[0], ws, w.tol, w.max_iters, stream)
-    return lambda: P.pararnn_lstm_solve_async(xd.u, xd.a, xd.c0, xd.h0, out[0], out[1], ws, w.tol,
-                                              w.max_iters, stream)
+class Step:
+    """One pass of the hot path on device-resident inputs, through the C ABI.
+    Records CUDA events on `stream` around the solve (and the adjoint)."""
+
+    def __init__(self, w, xd, dev, stream):
+        import nonlinear_rnn_newton_b200 as P
+        self.P, self.w, self.x, self.stream = P, w, xd, stream
+        ns = 1 if w.cell == "gru" else 2
+        self.out = [torch.empty((w.B, w.L, w.D), dtype=torch.float32, device=dev) for _ in range(ns)]
+        size = (P.pararnn_gru_workspace_size if w.cell == "gru" else P.pararnn_lstm_workspace_size)
+        self.ws = torch.empty(size(w.B, w.L, w.D), dtype=torch.uint8, device=dev)
+        self.adj = None
+        if w.train:
+            asize = (P.pararnn_gru_adjoint_workspace_size if w.cell == "gru"
+                     else P.pararnn_lstm_adjoint_workspace_size)
+            self.adj = {
+                "ws": torch.empty(asize(w.B, w.L, w.D), dtype=torch.uint8, device=dev),
+                "du": torch.empty((w.B, w.L, w.G, w.D), dtype=torch.float32, device=dev),
+                "da": torch.empty((w.G, w.D), dtype=torch.float32, device=dev),
+            }
+
+    def solve(self):
+        w, x, P = self.w, self.x, self.P
+        if w.cell == "gru":
+            P.pararnn_gru_solve_async(x.u, x.a, x.h0, self.out[0], self.ws, w.tol, w.max_iters, self.stream)
+        else:
+            P.pararnn_lstm_solve_async(x.u, x.a, x.c0, x.h0, self.out[0], self.out[1], self.ws, w.tol,
+                                       w.max_iters, self.stream)
+
+    def adjoint(self):
+        w, x, P, a = self.w, self.x, self.P, self.adj
+        if w.cell == "gru":
+            P.pararnn_gru_adjoint(x.u, x.a, x.h0, self.out[0], x.dh, du=a["du"], da=a["da"], want_dh0=False,
+                                  workspace=a["ws"], stream=self.stream)
+        else:
+            P.pararnn_lstm_adjoint(x.u, x.a, x.c0, x.h0, self.out[0], self.out[1], x.dh, du=a["du"],
+                                   da=a["da"], want_ds0=False, workspace=a["ws"], stream=self.stream)
+
+    def __call__(self, ev=None):
+        if ev is not None:
+            ev[0].record(self.stream)
+        self.solve()
+        if ev is not None:
+            ev[1].record(self.stream)
+        if self.adj is not None:
+            self.adjoint()
+            if ev is not None:
+                ev[2].record(self.stream)
+
+    def result(self):
+        return self.P.pararnn_read_result(self.ws, self.stream)
 
 
-def time_baselines(w, xd, out, stream, reps=5):
+def events(n, k):
+    return [[torch.cuda.Event(enable_timing=True) for _ in range(k)] for _ in range(n)]
+
+
+def time_baselines(w, xd, out, stream, dev, reps=5):
     """Device time of the two GPU baselines on the same input: the naive
     sequential step kernel (one thread per channel walks L) and one pass of the
-    plain diagonal linear scan (zero-weight GRU)."""
+    plain diagonal linear scan."""
     import nonlinear_rnn_newton_b200 as P
-    wsl = torch.empty(P.pararnn_linear_scan_workspace_size(w.B, w.L, w.D), dtype=torch.uint8, device=out.device)
+    wsl = torch.empty(P.pararnn_linear_scan_workspace_size(w.B, w.L, w.D), dtype=torch.uint8, device=dev)
+    es = 2 if w.u_dtype == "bf16" else 4
     res = {}
     for name, fn, nbytes in (
             ("sequential_gpu", lambda: P.pararnn_gru_sequential(xd.u, xd.a, xd.h0, out, stream=stream),
-             w.N * (w.G * (2 if w.u_dtype == "bf16" else 4) + 4)),
+             w.N * (w.G * es + 4)),
             ("linear_scan_gpu", lambda: P.pararnn_linear_scan(xd.u, xd.h0, out, wsl, stream=stream),
-             w.N * (2 * (2 if w.u_dtype == "bf16" else 4) + 4))):
+             w.N * (2 * es + 4))):
         for _ in range(2):
             fn()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -170,52 +270,161 @@ def time_baselines(w, xd, out, stream, reps=5):
         e1.record(stream)
         stream.synchronize()
         ms = e0.elapsed_time(e1) / reps
-        res[name] = {"ms": ms, "value": w.N / (ms * 1e-3), "unit": "tokens\u00b7channels/s",
-                     "gbs": nbytes / (ms * 1e-3) / 1e9}
+        res[name] = {"ms": ms, "value": w.N / (ms * 1e-3), "unit": UNIT, "gbs": nbytes / (ms * 1e-3) / 1e9}
     return res
 
 
-def cpu_oracle_sample(w, x, max_batches=1):
-    """Time the oracle's Newton solve on a bounded sample (the first batch rows)
-    of the workload.  Returns (tokens*channels/s, description, cores)."""
+def run_sweep(dev, stream, reps=10):
+    """The sequence-length sweep (B=1, D=2048): Newton solve, sequential GPU
+    kernel and linear scan at each L.  L <= 2048 fits in L2 (flagged)."""
+    import nonlinear_rnn_newton_b200 as P
+    peak, _ = hbm_peak()
+    out = []
+    for w in W.GRU_SWEEP:
+        xd = W.make_inputs(w, seed=0).to(dev)
+        st = Step(w, xd, dev, stream)
+        for _ in range(3):
+            st()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            st()
+        e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        r = st.result()
+        gbs = solve_bytes(w, r[1]) / (ms * 1e-3) / 1e9
+        base = time_baselines(w, xd, st.out[0], stream, dev)
+        out.append({"workload": w.name, "L": w.L, "ms": ms, "value": w.N / (ms * 1e-3), "iters": r[1],
+                    "status": r[0], "gbs": gbs, "frac": gbs / peak,
+                    "l2_resident": w.N * (w.G * 2 + 4) < 126e6,
+                    "sequential_gpu_ms": base["sequential_gpu"]["ms"],
+                    "linear_scan_gpu_ms": base["linear_scan_gpu"]["ms"]})
+        del st, xd
+        torch.cuda.empty_cache()
+    return out
+
+
+def oracle_sample(w, x, rows, chans):
+    """Sub-problem of the workload the oracle is timed on: the first `rows`
+    batch rows and `chans` channels (channels are independent, so this is the
+    same work per token*channel)."""
+    rows, chans = min(rows, w.B), min(chans, w.D)
+    u = x.u[:rows, :, :, :chans]
+    a = x.a[:, :chans]
+    h0 = None if x.h0 is None else x.h0[:rows, :chans]
+    dh = None if x.dh is None else x.dh[:rows, :, :chans]
+    return u, a, h0, dh, rows * w.L * chans
+
+
+def oracle_threads(w):
+    """Threads the oracle as it stands uses on this workload: its Newton solve
+    is one serial loop; its BPTT (training workload) runs OpenMP over channels."""
     import oracle
-    nb = min(max_batches, w.B)
-    u = x.u[:nb]
-    h0 = None if x.h0 is None else x.h0[:nb]
+    return oracle.max_threads() if w.train else 1
+
+
+def time_oracle(w, x, rows, chans, threads):
+    """Seconds of the oracle's Newton solve (plus BPTT for the training
+    workload) on the sample; the input widening to fp64 happens before the
+    clock starts."""
+    import numpy as np
+
+    import oracle
+    oracle.set_threads(threads)
+    u, a, h0, dh, n = oracle_sample(w, x, rows, chans)
+    u64, a64 = u.double().numpy(), a.double().numpy()
+    h064 = None if h0 is None else h0.double().numpy()
+    dh64 = None if dh is None else dh.double().numpy()
     t0 = time.perf_counter()
     if w.cell == "gru":
-        _, it, _, _, _ = oracle.gru_newton(u, x.a, h0, tol=w.tol, max_iters=w.max_iters)
+        h, it, _, _, _ = oracle.gru_newton(u64, a64, h064, tol=w.tol, max_iters=w.max_iters)
+        if dh64 is not None:
+            oracle.gru_bptt(u64, a64, h064, dh64)
     else:
-        _, _, it, _, _, _ = oracle.lstm_newton(u, x.a, None, h0, tol=w.tol, max_iters=w.max_iters)
+        c, h, it, _, _, _ = oracle.lstm_newton(u64, a64, None, h064, tol=w.tol, max_iters=w.max_iters)
+        if dh64 is not None:
+            oracle.lstm_bptt(u64, a64, None, h064, dh64)
     dt = time.perf_counter() - t0
-    n = nb * w.L * w.D
-    return n / dt, f"oracle Newton solve (fp64, serial C) on batch rows 0..{nb - 1} of the workload " \
-                   f"(B={nb}, L={w.L}, D={w.D}; {it} iterations), input conversion excluded", 1
+    assert np.isfinite(h).all()
+    what = "Newton solve" + (" + BPTT" if dh64 is not None else "")
+    how = "serial Newton" + (f", BPTT on {threads} OpenMP threads" if dh64 is not None else "")
+    desc = (f"oracle {what} (fp64 C, {how}) on batch rows 0..{min(rows, w.B) - 1}"
+            f", channels 0..{min(chans, w.D) - 1} of the workload (B={min(rows, w.B)}, L={w.L}, "
+            f"D={min(chans, w.D)}; {it} iterations); fp64 widening of the inputs excluded")
+    return n / dt, dt, desc
+
+
+def cpu_sample_shape(w):
+    """About 10-30 s of CPU work: the whole problem when it is cfg-1-sized,
+    else a slice of its channels."""
+    if w.N <= 40_000_000:
+        return w.B, w.D
+    return 1, max(128, min(w.D, 40_000_000 // (w.B * w.L)))
 
 
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    threads = oracle_threads(w)
     x = W.make_inputs(w, seed=0)
-    vals = []
-    desc = ""
+    # each step: one batch row (all channels) -- a bounded sample so that the
+    # whole run stays within minutes
+    chans = w.D if w.L * w.D <= 8_400_000 else max(128, 8_400_000 // w.L)
+    vals, desc = [], ""
     for i in range(args.warmup + args.steps):
-        v, desc, cores = cpu_oracle_sample(w, x, max_batches=1)
+        v, _, desc = time_oracle(w, x, 1, chans, threads)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value,
-        "unit": "tokens\u00b7channels/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * (w.L * w.D) / value, "higher_is_better": True, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name},
-        "cpu_baseline": {"value": value, "unit": "tokens\u00b7channels/s", "cores": 1, "kind": "oracle",
-                         "sample": desc},
-        "e2e": {"value": value, "unit": "tokens\u00b7channels/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "vs_baseline": None,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * (w.L * chans) / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_e2e(w, x, dev, stream, steps):
+    """The metric end to end through the public API: every step copies its
+    inputs from pinned host memory, runs the step and copies the states back
+    (all on one stream, timed with CUDA events)."""
+    hu = x.u.pin_memory()
+    ha = x.a.pin_memory()
+    hh0 = None if x.h0 is None else x.h0.pin_memory()
+    hdh = None if x.dh is None else x.dh.pin_memory()
+    du_ = torch.empty_like(hu, device=dev)
+    da_ = torch.empty_like(ha, device=dev)
+    dh0_ = None if hh0 is None else torch.empty_like(hh0, device=dev)
+    ddh_ = None if hdh is None else torch.empty_like(hdh, device=dev)
+    xe = W.Inputs(u=du_, a=da_, h0=dh0_, c0=None, dh=ddh_)
+    st = Step(w, xe, dev, stream)
+    hout = [torch.empty((w.B, w.L, w.D), dtype=torch.float32).pin_memory() for _ in st.out]
+    h2d = sum(t.numel() * t.element_size() for t in (hu, ha, hh0, hdh) if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+
+    def one():
+        with torch.cuda.stream(stream):
+            for d, h in ((du_, hu), (da_, ha), (dh0_, hh0), (ddh_, hdh)):
+                if h is not None:
+                    d.copy_(h, non_blocking=True)
+            st()
+            for o, ho in zip(st.out, hout):
+                ho.copy_(o, non_blocking=True)
+
+    one()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
 def main():
@@ -229,6 +438,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--baselines", type=int, default=1, help="also time the sequential GPU kernel and "
                     "the plain linear scan on the same input (GRU workloads)")
+    ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep (B=1, D=2048)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.BY_NAME[args.workload]
@@ -237,125 +447,103 @@ def main():
         run_reference(args, w)
         return
 
-    rank, world, local = dist_setup(args.gpus)
+    rank, world, local = dist_setup()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    import nonlinear_rnn_newton_b200 as P
     from nonlinear_rnn_newton_b200 import capi
 
     x = W.make_inputs(w, seed=rank)
     xd = x.to(dev)
-    ns = 1 if w.cell == "gru" else 2
-    out = [torch.empty((w.B, w.L, w.D), dtype=torch.float32, device=dev) for _ in range(ns)]
-    wsz = (P.pararnn_gru_workspace_size if w.cell == "gru" else P.pararnn_lstm_workspace_size)(w.B, w.L, w.D)
-    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
-    step = solve_fn(w, xd, out, ws, stream)
+    step = Step(w, xd, dev, stream)
 
     # warm-up (also validates the solve)
     for _ in range(args.warmup):
         step()
-    st, iters, resid, resid0 = P.pararnn_read_result(ws, stream)
+    st, iters, resid, resid0 = step.result()
     if st not in (0, 1):
         raise SystemExit(f"solve failed: status {st} ({capi.status_string(st)})")
 
-    # timed region: K back-to-back solves on one stream, CUDA events around each
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    # timed region: K back-to-back steps on one stream, CUDA events around
+    # each launch; inputs (> 126 MB) exceed L2, so no flush is needed
+    nev = 3 if w.train else 2
+    evs = events(args.steps, nev)
     barrier(world)
     torch.cuda.synchronize(dev)
     launches0 = capi.kernel_launch_count()
     with ClockSampler(local) as clk:
-        evs[0].record(stream)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
         for i in range(args.steps):
-            step()
-            evs[i + 1].record(stream)
+            step(evs[i])
+        t1.record(stream)
         stream.synchronize()
     launches = capi.kernel_launch_count() - launches0
     barrier(world)
     torch.cuda.synchronize(dev)
-    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
-    total_ms = evs[0].elapsed_time(evs[-1])
-    total_ms = max_over_ranks(total_ms, world)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
     ms_per_step = total_ms / args.steps
-    st2, iters2, resid2, _ = P.pararnn_read_result(ws, stream)
+    st2, iters2, resid2, _ = step.result()
+    solve_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    adj_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) if w.train else None
 
-    value = world * w.N / (ms_per_step * 1e-3)
+    value = job_value(w.N, world, ms_per_step)
     peak, peak_kind = hbm_peak()
-    algo = algorithmic_bytes(w, iters2)
-    mean_launch_ms = statistics.mean(per)
-    achieved = algo / (mean_launch_ms * 1e-3) / 1e9
+    # dominant kernel: the Newton solve (one launch per step)
+    algo = solve_bytes(w, iters2)
+    achieved = algo / (solve_ms * 1e-3) / 1e9
+    kname = "newton_solve_ws_kernel"
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": profile_traffic(kname, w.name), "peak_kind": peak_kind, "kernel": kname,
+                "algorithmic_bytes_per_launch": algo, "kernel_ms_mean": solve_ms}
+    adjoint = None
+    if w.train:
+        ab = adjoint_bytes(w)
+        adjoint = {"kernel_ms_mean": adj_ms, "algorithmic_bytes_per_launch": ab,
+                   "achieved": ab / (adj_ms * 1e-3) / 1e9, "frac": ab / (adj_ms * 1e-3) / 1e9 / peak}
 
-    # end to end through the public API with host buffers (pinned)
     e2e = None
     if args.e2e_steps > 0:
-        hu = x.u.pin_memory()
-        ha = x.a.pin_memory()
-        hh0 = None if x.h0 is None else x.h0.pin_memory()
-        hout = [torch.empty((w.B, w.L, w.D), dtype=torch.float32).pin_memory() for _ in range(ns)]
-        du_, da_ = torch.empty_like(xd.u), torch.empty_like(xd.a)
-        dh0_ = None if x.h0 is None else torch.empty_like(xd.h0)
-
-        class _X:
-            pass
-        xe = _X()
-        xe.u, xe.a, xe.h0, xe.c0 = du_, da_, dh0_, None
-        estep = solve_fn(w, xe, out, ws, stream)
-        h2d = hu.numel() * hu.element_size() + ha.numel() * 4 + (0 if hh0 is None else hh0.numel() * 4)
-        d2h = sum(o.numel() * 4 for o in hout)
-
-        def e2e_step():
-            with torch.cuda.stream(stream):
-                du_.copy_(hu, non_blocking=True)
-                da_.copy_(ha, non_blocking=True)
-                if hh0 is not None:
-                    dh0_.copy_(hh0, non_blocking=True)
-                estep()
-                for o, ho in zip(out, hout):
-                    ho.copy_(o, non_blocking=True)
-
-        e2e_step()
-        stream.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        stream.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
-        e2e = {"value": world * w.N / (ems * 1e-3), "unit": "tokens\u00b7channels/s", "ms_per_step": ems,
+        ems, h2d, d2h = run_e2e(w, x, dev, stream, args.e2e_steps)
+        ems = max_over_ranks(ems, world)
+        e2e = {"value": job_value(w.N, world, ems), "unit": UNIT, "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     baselines = None
     if args.baselines and w.cell == "gru":
-        baselines = time_baselines(w, xd, out[0], stream, reps=5)
+        baselines = time_baselines(w, xd, step.out[0], stream, dev)
+
+    sweep = run_sweep(dev, stream) if (args.sweep and rank == 0) else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = cpu_oracle_sample(w, x, max_batches=1)
-        cpu = {"value": v, "unit": "tokens\u00b7channels/s", "cores": cores, "kind": "oracle", "sample": desc}
+        threads = oracle_threads(w)
+        rows, chans = cpu_sample_shape(w)
+        v, secs, desc = time_oracle(w, x, rows, chans, threads)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": secs}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens\u00b7channels/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic",
-            "config": {"workload": w.name, "cell": w.cell, "B": w.B, "L": w.L, "D": w.D,
-                       "u_dtype": w.u_dtype, "tol": w.tol, "max_iters": w.max_iters,
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "cell": w.cell, "B": w.B, "L": w.L, "D": w.D, "u_dtype": w.u_dtype,
+                       "state_dtype": "f32", "tol": w.tol, "max_iters": w.max_iters,
+                       "step": "Newton solve" + (" + adjoint" if w.train else ""),
                        "l2": "inputs larger than L2 (gates + states > 126 MB); no flush",
-                       "per_rank": "independent problem, seed = rank"},
+                       "per_rank": "independent problem, seed = rank", "parallelism": f"replicas x{world}"},
             "iters": iters2, "residual": resid2, "status": st2,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": algo,
-                         "kernel_ms_mean": mean_launch_ms},
-            "per_iteration_frac": achieved / peak,
+            "roofline": roofline,
+            "adjoint": adjoint,
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "e2e": e2e,
             "cpu_baseline": cpu,
             "baselines": baselines,
+            "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
