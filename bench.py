@@ -389,41 +389,60 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(w, x, dev, stream, steps):
+def run_e2e(w, x, dev, steps, nbuf=2):
     """The metric end to end through the public API: every step copies its
-    inputs from pinned host memory, runs the step and copies the states back
-    (all on one stream, timed with CUDA events)."""
+    inputs from pinned host memory to the device, runs the step and copies
+    the states back to pinned host memory.  Steps are pipelined over `nbuf`
+    sets of device buffers and three streams (host-to-device copies, compute,
+    device-to-host copies), so that step i's copies overlap the compute of its
+    neighbours; every copy of every step stays inside the timed region, which
+    runs from the first copy of the first step to the last copy of the last."""
     hu = x.u.pin_memory()
     ha = x.a.pin_memory()
     hh0 = None if x.h0 is None else x.h0.pin_memory()
     hdh = None if x.dh is None else x.dh.pin_memory()
-    du_ = torch.empty_like(hu, device=dev)
-    da_ = torch.empty_like(ha, device=dev)
-    dh0_ = None if hh0 is None else torch.empty_like(hh0, device=dev)
-    ddh_ = None if hdh is None else torch.empty_like(hdh, device=dev)
-    xe = W.Inputs(u=du_, a=da_, h0=dh0_, c0=None, dh=ddh_)
-    st = Step(w, xe, dev, stream)
-    hout = [torch.empty((w.B, w.L, w.D), dtype=torch.float32).pin_memory() for _ in st.out]
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    sets = []
+    for _ in range(nbuf):
+        xe = W.Inputs(u=torch.empty_like(hu, device=dev), a=torch.empty_like(ha, device=dev),
+                      h0=None if hh0 is None else torch.empty_like(hh0, device=dev), c0=None,
+                      dh=None if hdh is None else torch.empty_like(hdh, device=dev))
+        st = Step(w, xe, dev, s_comp)
+        hout = [torch.empty((w.B, w.L, w.D), dtype=torch.float32).pin_memory() for _ in st.out]
+        sets.append((xe, st, hout, torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()))
     h2d = sum(t.numel() * t.element_size() for t in (hu, ha, hh0, hdh) if t is not None)
-    d2h = sum(t.numel() * t.element_size() for t in hout)
+    d2h = sum(t.numel() * t.element_size() for t in sets[0][2])
 
-    def one():
-        with torch.cuda.stream(stream):
-            for d, h in ((du_, hu), (da_, ha), (dh0_, hh0), (ddh_, hdh)):
+    def one(i):
+        xe, st, hout, ev_in, ev_comp, ev_out = sets[i % nbuf]
+        s_in.wait_event(ev_comp)  # this set's inputs are free once its last step has run
+        with torch.cuda.stream(s_in):
+            for d, h in ((xe.u, hu), (xe.a, ha), (xe.h0, hh0), (xe.dh, hdh)):
                 if h is not None:
                     d.copy_(h, non_blocking=True)
-            st()
+        ev_in.record(s_in)
+        s_comp.wait_event(ev_in)
+        s_comp.wait_event(ev_out)  # its outputs are free once they reached the host
+        st()
+        ev_comp.record(s_comp)
+        s_out.wait_event(ev_comp)
+        with torch.cuda.stream(s_out):
             for o, ho in zip(st.out, hout):
                 ho.copy_(o, non_blocking=True)
+        ev_out.record(s_out)
 
-    one()
-    stream.synchronize()
+    for i in range(nbuf):
+        one(i)
+    torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
-    stream.synchronize()
+    e0.record(s_in)
+    for i in range(steps):
+        one(i)
+    e1.record(s_out)
+    torch.cuda.synchronize(dev)
+    st0 = sets[0][1].result()
+    if st0[0] not in (0, 1):
+        raise SystemExit(f"end-to-end solve failed: status {st0[0]}")
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
@@ -435,7 +454,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.GRU.name, choices=sorted(W.BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--baselines", type=int, default=1, help="also time the sequential GPU kernel and "
                     "the plain linear scan on the same input (GRU workloads)")
     ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep (B=1, D=2048)")
@@ -506,7 +525,7 @@ def main():
     e2e = None
     if args.e2e_steps > 0:
         barrier(world)
-        ems, h2d, d2h = run_e2e(w, x, dev, stream, args.e2e_steps)
+        ems, h2d, d2h = run_e2e(w, x, dev, args.e2e_steps)
         ems = max_over_ranks(ems, world)
         e2e = {"value": job_value(w.N, world, ems), "unit": UNIT, "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
