@@ -46,12 +46,14 @@ constexpr int kWork = 2;    // per-tile work buffers (tiles n-1 and n are live)
 // A ticket hands out `group` consecutive chunks of one sequence; they run
 // back to back in one CTA, so only the first of them looks back across CTAs
 // (the others take their carry from the tile before, in registers).  This
-// shortens the chain of cross-CTA look-backs along a sequence, but the
-// chunks of a group then follow each other in time instead of running side
-// by side.  The 2x2-block cell, whose look-back steps are three times as
-// heavy, gains from groups of two; the diagonal cell does best without.
+// halves the chain of cross-CTA look-backs along a sequence.  The group's
+// second tile is prepared while the first one's look-back read is in flight
+// and its inclusive value is published together with the first one's, so the
+// chain advances two chunks per look-back.  (Longer groups would need the
+// control warp to wait for folds the compute warps can only produce after
+// the first tile's carry, so two is the longest that pays.)
 #ifndef PARARNN_WS_GROUP_GRU
-#define PARARNN_WS_GROUP_GRU 1
+#define PARARNN_WS_GROUP_GRU 2
 #endif
 #ifndef PARARNN_WS_GROUP_LSTM
 #define PARARNN_WS_GROUP_LSTM 2
@@ -235,6 +237,37 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 #pragma unroll
             for (int i = 0; i < kStages; ++i) tk[i] = __shfl_sync(0xffffffffu, tk[i], 0);
             float y_inc[NS][kV];  // inclusive value of the last tile handled here
+            // folds of work buffer `wkb` -> exclusive prefixes (in place); returns
+            // the tile's aggregate (the last inclusive prefix) in `run`
+            auto prefix = [&](int wkb, Map (&run)[kV]) {
+                float* agg = reinterpret_cast<float*>(work_at(wkb) + LY::off_agg);
+#pragma unroll
+                for (int j = 0; j < kV; ++j) run[j] = Map::identity();
+                for (int seg = 0; seg < CW; ++seg) {
+                    Map m[kV];
+#pragma unroll
+                    for (int i = 0; i < NC; ++i) {
+                        float* row = agg + (i * CW + seg) * kDc + lane * kV;
+                        F4 v = load4(row);
+                        float v4[kV];
+#pragma unroll
+                        for (int j = 0; j < kV; ++j) {
+                            m[j].set(i, v.v[j]);
+                            v4[j] = run[j].get(i);
+                        }
+                        store4(row, v4);
+                    }
+#pragma unroll
+                    for (int j = 0; j < kV; ++j) run[j] = compose(m[j], run[j]);
+                }
+            };
+            // A group's second tile is prepared while its first tile's look-back
+            // read is in flight: its prefixes are computed (run_pre) and, as soon
+            // as the first tile's carry is known, its inclusive value is
+            // published, so that the next group's look-back does not wait for
+            // this CTA to reach it.
+            bool pre_done = false;  // the next tile's prefixes are computed (run_pre)
+            Map run_pre[kV];
             for (int n = 0;; ++n) {
                 const int s = n % kStages, wb = n % kWork;
                 int ticket = tk[0];
@@ -259,52 +292,51 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 #pragma unroll
                     for (int j = 0; j < kV; ++j) init[q][j] = x.v[j];
                 }
-                unsigned char* wk = work_at(wb);
-                float* agg = reinterpret_cast<float*>(wk + LY::off_agg);
-                float* car = reinterpret_cast<float*>(wk + LY::off_carry);
-                bool ok = mbar_wait_bounded(&bar_aggr[wb], uint32_t(n / kWork) & 1u, err, p.wait_ns);
-                // folds -> exclusive prefixes (in place); the last inclusive
-                // prefix is the tile's aggregate
+                float* car = reinterpret_cast<float*>(work_at(wb) + LY::off_carry);
+                bool ok = true;
                 Map run[kV];
+                if (local && pre_done) {
 #pragma unroll
-                for (int j = 0; j < kV; ++j) run[j] = Map::identity();
-                for (int seg = 0; seg < CW; ++seg) {
-                    Map m[kV];
-#pragma unroll
-                    for (int i = 0; i < NC; ++i) {
-                        float* row = agg + (i * CW + seg) * kDc + lane * kV;
-                        F4 v = load4(row);
-                        float v4[kV];
-#pragma unroll
-                        for (int j = 0; j < kV; ++j) {
-                            m[j].set(i, v.v[j]);
-                            v4[j] = run[j].get(i);
-                        }
-                        store4(row, v4);
-                    }
-#pragma unroll
-                    for (int j = 0; j < kV; ++j) run[j] = compose(m[j], run[j]);
+                    for (int j = 0; j < kV; ++j) run[j] = run_pre[j];
+                } else {
+                    ok = mbar_wait_bounded(&bar_aggr[wb], uint32_t(n / kWork) & 1u, err, p.wait_ns);
+                    prefix(wb, run);
                 }
                 float y[NS][kV];
                 if (local) {
+                    // carry = inclusive value of the group's previous tile; this
+                    // tile's inclusive value was published already if pre_done
 #pragma unroll
                     for (int q = 0; q < NS; ++q)
 #pragma unroll
                         for (int j = 0; j < kV; ++j) y[q][j] = y_inc[q][j];
-                }
-                // the tile's inclusive value, kept for the next tile of the group
 #pragma unroll
-                for (int j = 0; j < kV; ++j) {
-                    float x[NS], z[NS];
+                    for (int j = 0; j < kV; ++j) {
+                        float x[NS], z[NS];
 #pragma unroll
-                    for (int q = 0; q < NS; ++q) x[q] = y[q][j];
-                    apply(run[j], x, z);
+                        for (int q = 0; q < NS; ++q) x[q] = y[q][j];
+                        apply(run[j], x, z);
 #pragma unroll
-                    for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
-                }
-                if (local) {
-                    publish_inclusive<Map, NS>(p.desc, ticket, k, y_inc, lane);
+                        for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
+                    }
+                    if (!pre_done) publish_inclusive<Map, NS>(p.desc, ticket, k, y_inc, lane);
+                    pre_done = false;
                 } else {
+                    // the group's next tile, if it is the next in the ring: its
+                    // prefixes now, while the look-back read is in flight
+                    if (kGroup > 1) {
+                        const int n1 = n + 1, s1 = n1 % kStages;
+                        int t1 = tk[0];
+#pragma unroll
+                        for (int i = 1; i < kStages; ++i)
+                            if (s1 == i) t1 = tk[i];
+                        if (t1 < p.n_tiles && t1 == ticket + BS && ((c + 1) % kGroup) != 0) {
+                            ok = mbar_wait_bounded(&bar_aggr[n1 % kWork], uint32_t(n1 / kWork) & 1u, err, p.wait_ns) &&
+                                 ok;
+                            prefix(n1 % kWork, run_pre);
+                            pre_done = true;
+                        }
+                    }
                     ok = lookback<Map, NS>(ticket, BS, c > 0, k, run, init, y, p.desc, lane, err, p.wait_ns, pr) && ok;
 #pragma unroll
                     for (int j = 0; j < kV; ++j) {
@@ -314,6 +346,20 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                         apply(run[j], x, z);
 #pragma unroll
                         for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
+                    }
+                    if (pre_done) {
+                        // the next tile's inclusive value, published right away
+                        float yn[NS][kV];
+#pragma unroll
+                        for (int j = 0; j < kV; ++j) {
+                            float x[NS], z[NS];
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) x[q] = y_inc[q][j];
+                            apply(run_pre[j], x, z);
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) yn[q][j] = z[q];
+                        }
+                        publish_inclusive<Map, NS>(p.desc, ticket + BS, k, yn, lane);
                     }
                 }
 #pragma unroll
