@@ -281,9 +281,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 // inside a group the tile before ran here: its inclusive value
                 // (y_inc) is this tile's carry
                 const bool local = (c % kGroup) != 0;
-                // first look-back read, in flight while the folds are composed
                 LookbackProbe<Map, NS> pr;
-                if (c > 0 && !local) lookback_probe(pr, ticket - BS, p.desc, lane);
+
                 float init[NS][kV];
 #pragma unroll
                 for (int q = 0; q < NS; ++q) {
@@ -300,6 +299,9 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     for (int j = 0; j < kV; ++j) run[j] = run_pre[j];
                 } else {
                     ok = mbar_wait_bounded(&bar_aggr[wb], uint32_t(n / kWork) & 1u, err, p.wait_ns);
+                    // first look-back read, in flight while the folds are composed
+                    // (issued only now, so that it sees predecessors as late as possible)
+                    if (c > 0 && !local) lookback_probe(pr, ticket - BS, p.desc, lane);
                     prefix(wb, run);
                 }
                 float y[NS][kV];
