@@ -49,10 +49,18 @@ struct AdjointLayout {
     static constexpr size_t s_bytes = size_t(Lc) * kDc * sizeof(float);
     static constexpr size_t scan_floats = size_t(NC) * kWarps * kScanPad;
     static constexpr size_t red_floats = size_t(kWarps) * G * kDc;
+    // stage: gates | states [NS][Lc][kDc] | upstream [NS][Lc][kDc]
     static constexpr size_t off_u = 0;
-    static constexpr size_t off_s = off_u + u_bytes;           // states [NS][Lc][kDc]
-    static constexpr size_t off_g = off_s + NS * s_bytes;      // upstream [NS][Lc][kDc]
-    static constexpr size_t off_scan = off_g + NS * s_bytes;   // scan scratch, reused for the da reduction
+    static constexpr size_t off_s = off_u + u_bytes;
+    static constexpr size_t off_g = off_s + NS * s_bytes;
+    static constexpr size_t stage_bytes = off_g + NS * s_bytes;
+    // after the stages: scan scratch (reused for the da reduction), tile
+    // aggregate, carry, two mbarriers and the stages' tickets
+    static constexpr size_t rest_bytes = 4 * (scan_floats > red_floats ? scan_floats : red_floats) +
+                                         size_t(NC) * kDc * 4 + size_t(NS) * kDc * 4 + 64;
+    // two stages (the next tile loads while this one is swept) where they fit
+    static constexpr int kStg = 2 * stage_bytes + rest_bytes <= 232448 ? 2 : 1;
+    static constexpr size_t off_scan = kStg * stage_bytes;
     static constexpr size_t off_tagg = off_scan + 4 * (scan_floats > red_floats ? scan_floats : red_floats);
     static constexpr size_t off_carry = off_tagg + size_t(NC) * kDc * 4;
     static constexpr size_t off_misc = off_carry + size_t(NS) * kDc * 4;
@@ -71,15 +79,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     using Map = typename Cell::Map;
     constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc;
 
+    constexpr int NSTG = LY::kStg;
     extern __shared__ __align__(128) unsigned char smem[];
-    UT* su = reinterpret_cast<UT*>(smem + LY::off_u);
-    float* ss = reinterpret_cast<float*>(smem + LY::off_s);
-    float* sg = reinterpret_cast<float*>(smem + LY::off_g);
     float* scan = reinterpret_cast<float*>(smem + LY::off_scan);
     float* tagg = reinterpret_cast<float*>(smem + LY::off_tagg);
     float* scarry = reinterpret_cast<float*>(smem + LY::off_carry);
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + LY::off_misc);
-    int* s_int = reinterpret_cast<int*>(smem + LY::off_misc + 16);
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + LY::off_misc);  // [NSTG]
+    int* s_int = reinterpret_cast<int*>(smem + LY::off_misc + 16);      // [0..1] flags, [2..3] tickets
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     WsHeader* hdr = p.hdr;
@@ -87,23 +93,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long D = p.D, L = p.L;
     const int BS = int(p.B) * p.S;
 
+    // thread 0: ticket t's loads into stage i (no-op for an invalid ticket)
+    auto issue = [&](int t, int i) {
+        s_int[2 + i] = t;
+        if (t >= p.n_tiles) return;
+        const int cc = p.n_chunks - 1 - t / BS, rr = t % BS;
+        const int bb = rr / p.S, dd = (rr - bb * p.S) * kDc, ll = cc * Lc;
+        unsigned char* st = smem + i * LY::stage_bytes;
+        fence_proxy_async_shared();
+        uint32_t bytes = uint32_t(LY::u_bytes + NS * LY::s_bytes);
+#pragma unroll
+        for (int q = 0; q < NS; ++q)
+            if (p.has_g[q]) bytes += uint32_t(LY::s_bytes);
+        mbar_arrive_expect_tx(&mbar[i], bytes);
+        tma_load_4d(st + LY::off_u, &tm_u, dd, 0, ll, bb, &mbar[i]);
+        tma_load_3d(st + LY::off_s, &tm_s0, dd, ll, bb, &mbar[i]);
+        if (NS == 2) tma_load_3d(st + LY::off_s + LY::s_bytes, &tm_s1, dd, ll, bb, &mbar[i]);
+        if (p.has_g[0]) tma_load_3d(st + LY::off_g, &tm_g0, dd, ll, bb, &mbar[i]);
+        if (NS == 2 && p.has_g[NS - 1]) tma_load_3d(st + LY::off_g + LY::s_bytes, &tm_g1, dd, ll, bb, &mbar[i]);
+    };
+    auto take = [&]() {
+        const int t = int(atomicAdd(&hdr->tick[0], 1u));
+        return error_raised(err) ? INT_MAX : t;
+    };
+
     if (tid == 0) {
-        mbar_init(mbar, 1);
+        for (int i = 0; i < NSTG; ++i) mbar_init(&mbar[i], 1);
         fence_mbar_init();
         prefetch_tensormap(&tm_u);
+        // tickets are taken in order and handled in order, tile n in stage n % NSTG
+        for (int i = 0; i < NSTG; ++i) issue(take(), i);
     }
     __syncthreads();
-    uint32_t phase = 0;
 
-    for (;;) {
-        if (tid == 0) {
-            int t = int(atomicAdd(&hdr->tick[0], 1u));
-            if (error_raised(err)) t = INT_MAX;
-            s_int[0] = t;
+    for (int n = 0;; ++n) {
+        // the tile before this one is finished: its stage takes tile n+NSTG-1
+        if (n >= 1 && tid == 0) {
+            const int last = s_int[2 + (n - 1) % NSTG];
+            issue(last < p.n_tiles ? take() : INT_MAX, (n + NSTG - 1) % NSTG);
         }
         __syncthreads();
-        const int ticket = s_int[0];
+        const int stg = n % NSTG;
+        const int ticket = s_int[2 + stg];
         if (ticket >= p.n_tiles) break;
+        UT* su = reinterpret_cast<UT*>(smem + stg * LY::stage_bytes + LY::off_u);
+        float* ss = reinterpret_cast<float*>(smem + stg * LY::stage_bytes + LY::off_s);
+        float* sg = reinterpret_cast<float*>(smem + stg * LY::stage_bytes + LY::off_g);
         // reverse chunk order: the last chunk gets the first tickets
         const int c = p.n_chunks - 1 - ticket / BS;
         const int rem = ticket % BS;
@@ -112,19 +147,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int l0 = c * Lc;
         const int d0 = sl * kDc;
 
-        if (tid == 0) {
-            fence_proxy_async_shared();
-            uint32_t bytes = uint32_t(LY::u_bytes + NS * LY::s_bytes);
-#pragma unroll
-            for (int q = 0; q < NS; ++q)
-                if (p.has_g[q]) bytes += uint32_t(LY::s_bytes);
-            mbar_arrive_expect_tx(mbar, bytes);
-            tma_load_4d(su, &tm_u, d0, 0, l0, b, mbar);
-            tma_load_3d(ss, &tm_s0, d0, l0, b, mbar);
-            if (NS == 2) tma_load_3d(ss + Lc * kDc, &tm_s1, d0, l0, b, mbar);
-            if (p.has_g[0]) tma_load_3d(sg, &tm_g0, d0, l0, b, mbar);
-            if (NS == 2 && p.has_g[NS - 1]) tma_load_3d(sg + Lc * kDc, &tm_g1, d0, l0, b, mbar);
-        }
         const int dch = d0 + lane * kV;
         const bool chv = dch < D;
         float wv[G][kV];
@@ -149,8 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < kV; ++j) halo[q][j] = x.v[j];
         }
-        if (!mbar_wait_bounded(mbar, phase, err, p.wait_ns)) s_int[0] = INT_MAX;
-        phase ^= 1u;
+        (void)mbar_wait_bounded(&mbar[stg], uint32_t(n / NSTG) & 1u, err, p.wait_ns);
 
         const int r0 = w * T;
         // element access helpers (row within the tile)
@@ -235,7 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) s_int[1] = ok ? 0 : 1;
         }
         __syncthreads();
-        if (s_int[1]) break;
+        if (s_int[1]) {
+            // look-back gave up: let the next tile's copy land before leaving
+            if (NSTG > 1 && tid == 0 && s_int[2 + (n + 1) % NSTG] < p.n_tiles)
+                (void)mbar_wait_bounded(&mbar[(n + 1) % NSTG], uint32_t((n + 1) / NSTG) & 1u, err, p.wait_ns);
+            break;
+        }
 
         // Sweep 2 (reverse): lambda, du, da partials, mu
         float dacc[G][kV];
