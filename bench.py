@@ -1,7 +1,7 @@
 """Benchmark of the ParaRNN Newton solve on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-cpu-baseline] [--sweep]
+                    [--workload NAME] [--no-cpu-baseline] [--sweep] [--decode]
 
 A step is one pass of the whole hot path over the workload through the C ABI:
 one full Newton solve (every iteration until convergence, the convergence
@@ -305,6 +305,51 @@ def run_sweep(dev, stream, reps=10):
     return out
 
 
+def run_decode(dev, stream, T=256, reps=5):
+    """Decode steps (one recurrence step for B sequences, state updated in
+    place) at the solve workloads' width D=1024, bf16 gates: T steps captured
+    in one CUDA graph, timed over `reps` replays; per step one kernel launch."""
+    import nonlinear_rnn_newton_b200 as P
+    out = []
+    for cell in ("gru", "lstm"):
+        for B in (8, 256):
+            w = W.custom(cell, B, T, 1024, "bf16", h0_std=0.1)
+            x = W.make_inputs(w, seed=0)
+            u = x.u.transpose(0, 1).contiguous().to(dev)  # [T, B, G, D]: one contiguous slab per step
+            a = x.a.to(dev)
+            h = torch.zeros((B, w.D), device=dev)
+            c = torch.zeros((B, w.D), device=dev)
+
+            def steps():
+                for t in range(T):
+                    if cell == "gru":
+                        P.pararnn_gru_step(u[t], a, h, h, stream=stream)
+                    else:
+                        P.pararnn_lstm_step(u[t], a, c, h, c, h, stream=stream)
+
+            with torch.cuda.stream(stream):
+                steps()  # warm up outside the capture
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    steps()
+                for _ in range(2):
+                    g.replay()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / (reps * T)
+            ns = 1 if cell == "gru" else 2
+            nbytes = B * w.D * (w.G * 2 + 8 * ns) + w.G * w.D * 4  # gates, state read + write, weights
+            out.append({"cell": cell, "B": B, "D": w.D, "us_per_step": round(us, 3),
+                        "tokens_per_s": B / (us * 1e-6), "gbs": nbytes / (us * 1e-6) / 1e9,
+                        "launches_per_step": 1})
+            del g, u
+    return out
+
+
 def oracle_sample(w, x, rows, chans):
     """Sub-problem of the workload the oracle is timed on: the first `rows`
     batch rows and `chans` channels (channels are independent, so this is the
@@ -458,6 +503,7 @@ def main():
     ap.add_argument("--baselines", type=int, default=1, help="also time the sequential GPU kernel and "
                     "the plain linear scan on the same input (GRU workloads)")
     ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep (B=1, D=2048)")
+    ap.add_argument("--decode", action="store_true", help="add the decode-step timings (CUDA graph of steps)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.BY_NAME[args.workload]
@@ -535,6 +581,7 @@ def main():
         baselines = time_baselines(w, xd, step.out[0], stream, dev)
 
     sweep = run_sweep(dev, stream) if (args.sweep and rank == 0) else None
+    decode = run_decode(dev, stream) if (args.decode and rank == 0) else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -563,6 +610,7 @@ def main():
             "cpu_baseline": cpu,
             "baselines": baselines,
             "sweep": sweep,
+            "decode": decode,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -218,6 +218,31 @@ PARARNN_API pararnn_status pararnn_lstm_adjoint(const void* u, pararnn_dtype u_d
                                     int64_t D, void* workspace, size_t workspace_bytes,
                                     pararnn_stream_t stream);
 
+/* ----------------------------------------------------------- decode step */
+
+/* One recurrence step for B sequences at once, the token-by-token generation
+ * that "Por que RNN ainda importa" credits RNNs with (cost per token fixed,
+ * whatever the context length): s_next = f(s_prev, u) with the cells of the
+ * solves above.
+ *   u       [B][G][D] gate pre-activations of this step (G = 3: z, r, c for
+ *           the GRU; G = 4: i, f, o, g for the LSTM), bf16 or fp32
+ *   a       [G][D] diagonal recurrence weights, fp32
+ *   *_prev  [B][D] current state, fp32; NULL = zeros
+ *   *_next  [B][D] next state, fp32, written in full
+ * All device pointers, 16-byte aligned; D a multiple of 8.  An output may be
+ * the very buffer of its own previous state (update in place); any other
+ * overlap between outputs and inputs, or between c_next and h_next, is
+ * refused with PARARNN_ERR_INVALID_ARG before any launch.  One kernel launch,
+ * asynchronous on `stream`, capturable in a CUDA graph; the library keeps no
+ * state between calls. */
+PARARNN_API pararnn_status pararnn_gru_step(const void* u, pararnn_dtype u_dtype, const float* a,
+                                            const float* h_prev, float* h_next, int64_t B,
+                                            int64_t D, pararnn_stream_t stream);
+PARARNN_API pararnn_status pararnn_lstm_step(const void* u, pararnn_dtype u_dtype, const float* a,
+                                             const float* c_prev, const float* h_prev,
+                                             float* c_next, float* h_next, int64_t B, int64_t D,
+                                             pararnn_stream_t stream);
+
 /* ------------------------------------------------------------- baselines */
 
 /* Naive sequential application ("O compromisso que SSMs fizeram": one step

@@ -19,6 +19,7 @@ __all__ = [
     "pararnn_gru_solve_async",
     "pararnn_gru_solve_noalloc",
     "pararnn_gru_solve_noalloc_max_scratch",
+    "pararnn_gru_step",
     "pararnn_gru_workspace_size",
     "pararnn_linear_scan",
     "pararnn_linear_scan_workspace_size",
@@ -27,6 +28,7 @@ __all__ = [
     "pararnn_lstm_sequential",
     "pararnn_lstm_solve",
     "pararnn_lstm_solve_async",
+    "pararnn_lstm_step",
     "pararnn_lstm_workspace_size",
     "pararnn_read_result",
     "pararnn_selftest_wait_timeout",

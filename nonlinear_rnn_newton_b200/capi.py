@@ -71,6 +71,8 @@ SIGNATURES = {
                                    _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "pararnn_gru_sequential": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "pararnn_lstm_sequential": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "pararnn_gru_step": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _vp]),
+    "pararnn_lstm_step": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp]),
     "pararnn_linear_scan": (_st, [_vp, _st, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "pararnn_status_string": (ctypes.c_char_p, [_st]),
     "pararnn_last_error": (ctypes.c_char_p, []),
@@ -349,6 +351,30 @@ def pararnn_lstm_adjoint(u, a, c0, h0, c, h, dh, dc=None, du=None, da=None, dc0=
                                   _ptr(ws), ws.numel(), _stream(dev, stream))
     _check(st, allow=(OK,))
     return du, da, dc0, dh0
+
+
+# ------------------------------------------------------------- decode step
+
+def pararnn_gru_step(u, a, h_prev=None, h_next=None, stream=None):
+    """One step for B sequences: u [B, 3, D], h_prev [B, D] (None = zeros).
+    h_next may be h_prev itself (in place); a new tensor if None."""
+    B, G, D = u.shape
+    h_next = h_next if h_next is not None else torch.empty((B, D), dtype=torch.float32, device=u.device)
+    st = lib.pararnn_gru_step(_ptr(u), _dtype_code(u), _ptr(a), _ptr(h_prev), _ptr(h_next), B, D,
+                              _stream(u.device, stream))
+    _check(st, allow=(OK,))
+    return h_next
+
+
+def pararnn_lstm_step(u, a, c_prev=None, h_prev=None, c_next=None, h_next=None, stream=None):
+    """One step for B sequences: u [B, 4, D], c_prev, h_prev [B, D] (None = zeros)."""
+    B, G, D = u.shape
+    c_next = c_next if c_next is not None else torch.empty((B, D), dtype=torch.float32, device=u.device)
+    h_next = h_next if h_next is not None else torch.empty((B, D), dtype=torch.float32, device=u.device)
+    st = lib.pararnn_lstm_step(_ptr(u), _dtype_code(u), _ptr(a), _ptr(c_prev), _ptr(h_prev), _ptr(c_next),
+                               _ptr(h_next), B, D, _stream(u.device, stream))
+    _check(st, allow=(OK,))
+    return c_next, h_next
 
 
 # --------------------------------------------------------------- baselines

@@ -20,6 +20,7 @@
 #include "newton.cuh"
 #include "newton_ws.cuh"
 #include "sequential.cuh"
+#include "decode.cuh"
 #include "adjoint.cuh"
 #include "linear_scan.cuh"
 
@@ -650,6 +651,50 @@ pararnn_status noalloc_scratch(void** out)
     return PARARNN_OK;
 }
 
+// decode step: shape and aliasing checks, launch
+pararnn_status check_step_shape(int64_t B, int64_t D)
+{
+    if (B < 1 || D < 1) return fail(PARARNN_ERR_INVALID_ARG, "B, D must be >= 1 (got %lld, %lld)", (long long)B,
+                                    (long long)D);
+    if (D % 8 != 0) return fail(PARARNN_ERR_UNSUPPORTED, "D must be a multiple of 8 (got %lld)", (long long)D);
+    if ((double)B * (double)D * 16.0 >= 1099511627776.0) return fail(PARARNN_ERR_INVALID_ARG, "B*D too large");
+    return PARARNN_OK;
+}
+
+// do the n-float ranges at x and y share a byte?
+bool overlap(const float* x, const float* y, long long n)
+{
+    if (!x || !y) return false;
+    const uintptr_t x0 = reinterpret_cast<uintptr_t>(x), y0 = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t len = uintptr_t(n) * 4;
+    return x0 < y0 + len && y0 < x0 + len;
+}
+
+// an output may be its own previous state; any other overlap is refused
+pararnn_status check_alias(const float* in, const float* out, long long n, const char* name)
+{
+    if (in != out && overlap(in, out, n))
+        return fail(PARARNN_ERR_INVALID_ARG, "%s overlaps an input without being its own previous state", name);
+    return PARARNN_OK;
+}
+
+template <class Cell>
+pararnn_status launch_step(const void* u, pararnn_dtype u_dtype, const float* a, const float* p0, const float* p1,
+                           float* n0, float* n1, int64_t B, int64_t D, cudaStream_t st)
+{
+    const long long n4 = (long long)B * D / 4;
+    if (n4 == 0) return PARARNN_OK;
+    const dim3 block(256), grid(unsigned((n4 + 255) / 256));
+    if (u_dtype == PARARNN_BF16)
+        decode_step_kernel<Cell, uint16_t>
+            <<<grid, block, 0, st>>>(static_cast<const uint16_t*>(u), a, p0, p1, n0, n1, B, D);
+    else
+        decode_step_kernel<Cell, float><<<grid, block, 0, st>>>(static_cast<const float*>(u), a, p0, p1, n0, n1, B, D);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -804,6 +849,46 @@ pararnn_status pararnn_lstm_sequential(const void* u, pararnn_dtype u_dtype, con
     CUDA_TRY(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return PARARNN_OK;
+}
+
+// ---------------------------------------------------------- decode step
+
+pararnn_status pararnn_gru_step(const void* u, pararnn_dtype u_dtype, const float* a, const float* h_prev,
+                                float* h_next, int64_t B, int64_t D, pararnn_stream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(u_dtype));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(h_prev, "h_prev", false));
+    TRY(check_ptr(h_next, "h_next", true));
+    TRY(check_step_shape(B, D));
+    TRY(check_alias(h_prev, h_next, (long long)B * D, "h_next"));
+    return launch_step<GruCell>(u, u_dtype, a, h_prev, nullptr, h_next, nullptr, B, D,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_lstm_step(const void* u, pararnn_dtype u_dtype, const float* a, const float* c_prev,
+                                 const float* h_prev, float* c_next, float* h_next, int64_t B, int64_t D,
+                                 pararnn_stream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(u_dtype));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(c_prev, "c_prev", false));
+    TRY(check_ptr(h_prev, "h_prev", false));
+    TRY(check_ptr(c_next, "c_next", true));
+    TRY(check_ptr(h_next, "h_next", true));
+    TRY(check_step_shape(B, D));
+    const long long n = (long long)B * D;
+    TRY(check_alias(c_prev, c_next, n, "c_next"));
+    TRY(check_alias(h_prev, h_next, n, "h_next"));
+    if (overlap(h_prev, c_next, n)) return fail(PARARNN_ERR_INVALID_ARG, "c_next overlaps h_prev");
+    if (overlap(c_prev, h_next, n)) return fail(PARARNN_ERR_INVALID_ARG, "h_next overlaps c_prev");
+    if (overlap(c_next, h_next, n)) return fail(PARARNN_ERR_INVALID_ARG, "c_next and h_next overlap");
+    return launch_step<LstmCell>(u, u_dtype, a, c_prev, h_prev, c_next, h_next, B, D,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t pararnn_linear_scan_workspace_size(int64_t B, int64_t L, int64_t D) { return linear_scan_ws_bytes(B, L, D); }

@@ -101,12 +101,34 @@ def test_argument_checks_before_any_gpu_work(capi):
     assert lib.pararnn_selftest_wait_timeout(5, 10, 256, 16384, None) == E.ERR_INVALID_ARG
 
 
+def test_decode_step_checks(capi):
+    """The decode step refuses bad shapes, pointers and partial overlaps
+    before any launch; an output that is its own previous state passes."""
+    E, lib = capi, capi.lib
+    gru = lambda u=16, a=16, hp=None, hn=4096, B=1, D=16: lib.pararnn_gru_step(u, 1, a, hp, hn, B, D, None)
+    assert gru(D=12) == E.ERR_UNSUPPORTED
+    assert gru(B=0) == E.ERR_INVALID_ARG
+    assert gru(u=None) == E.ERR_INVALID_ARG
+    assert gru(hn=4104) == E.ERR_INVALID_ARG  # misaligned
+    assert gru(hp=4096 - 48, hn=4096) == E.ERR_INVALID_ARG  # ranges of 64 bytes overlap
+    assert "overlaps" in capi.last_error()
+    lstm = lambda cp=None, hp=None, cn=4096, hn=8192, D=16: lib.pararnn_lstm_step(16, 1, 16, cp, hp, cn, hn, 1, D,
+                                                                                   None)
+    assert lstm(cn=8192, hn=8192) == E.ERR_INVALID_ARG
+    assert lstm(hp=4096) == E.ERR_INVALID_ARG  # h_prev is c_next
+    assert lstm(cp=8192) == E.ERR_INVALID_ARG  # c_prev is h_next
+    assert lstm(D=4) == E.ERR_UNSUPPORTED
+
+
 def test_valid_arguments_without_gpu_report_cuda_error(capi):
     import torch
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _solve(capi) == capi.ERR_CUDA
     assert capi.last_error()
+    # in place (the output is its own previous state): accepted, then no device
+    assert capi.lib.pararnn_gru_step(16, 1, 16, 4096, 4096, 1, 16, None) == capi.ERR_CUDA
+    assert capi.lib.pararnn_lstm_step(16, 1, 16, 4096, 8192, 4096, 8192, 1, 16, None) == capi.ERR_CUDA
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
