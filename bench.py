@@ -1,7 +1,7 @@
 """Benchmark of the ParaRNN Newton solve on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-cpu-baseline] [--sweep] [--decode]
+                    [--workload NAME] [--no-cpu-baseline] [--sweep] [--decode] [--cells]
 
 A step is one pass of the whole hot path over the workload through the C ABI:
 one full Newton solve (every iteration until convergence, the convergence
@@ -17,6 +17,7 @@ Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle on a
 bounded sample of the same workload instead (the reference arm; rank 0 only).
 """
 import argparse
+import itertools
 import hashlib
 import json
 import os
@@ -350,6 +351,45 @@ def run_decode(dev, stream, T=256, reps=5):
     return out
 
 
+def run_cells(dev, stream, reps=5):
+    """User-written cells (the GRU and LSTM sources of example_cells, compiled
+    at run time) on the solve workloads, beside the built-in kernels."""
+    import nonlinear_rnn_newton_b200 as P
+    from nonlinear_rnn_newton_b200 import example_cells
+    peak, _ = hbm_peak()
+    out = []
+    for (w, src), flags in itertools.product(((W.GRU, example_cells.GRU), (W.LSTM, example_cells.LSTM)), (0, 1)):
+        ns = 1 if w.cell == "gru" else 2
+        with torch.cuda.device(dev):
+            cell = P.pararnn_cell_create(src, w.G, ns, flags)
+        x = W.make_inputs(w, seed=0).to(dev)
+        s0 = torch.zeros((ns, w.B, w.D), device=dev)
+        if x.h0 is not None:
+            s0[ns - 1] = x.h0
+        s = torch.empty((ns, w.B, w.L, w.D), device=dev)
+        ws = torch.empty(P.pararnn_cell_workspace_size(cell, x.u.dtype, w.B, w.L, w.D), dtype=torch.uint8,
+                         device=dev)
+        run = lambda: P.pararnn_cell_solve_async(cell, x.u, x.a, s0, s, ws, tol=w.tol, max_iters=w.max_iters,
+                                                 stream=stream)
+        for _ in range(3):
+            run()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            run()
+        e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        r = P.pararnn_read_result(ws, stream)
+        gbs = solve_bytes(w, r[1]) / (ms * 1e-3) / 1e9
+        out.append({"workload": w.name, "cell": f"{w.cell} (user source)", "fast_math": bool(flags),
+                    "compute_warps": P.pararnn_cell_compute_warps(cell, x.u.dtype), "ms": round(ms, 4), "iters": r[1],
+                    "status": r[0], "value": w.N / (ms * 1e-3), "gbs": gbs, "frac": gbs / peak})
+        del cell, ws, s, x
+        torch.cuda.empty_cache()
+    return out
+
+
 def oracle_sample(w, x, rows, chans):
     """Sub-problem of the workload the oracle is timed on: the first `rows`
     batch rows and `chans` channels (channels are independent, so this is the
@@ -504,6 +544,7 @@ def main():
                     "the plain linear scan on the same input (GRU workloads)")
     ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep (B=1, D=2048)")
     ap.add_argument("--decode", action="store_true", help="add the decode-step timings (CUDA graph of steps)")
+    ap.add_argument("--cells", action="store_true", help="add the runtime-compiled user cells (GRU, LSTM sources)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.BY_NAME[args.workload]
@@ -582,6 +623,7 @@ def main():
 
     sweep = run_sweep(dev, stream) if (args.sweep and rank == 0) else None
     decode = run_decode(dev, stream) if (args.decode and rank == 0) else None
+    cells = run_cells(dev, stream) if (args.cells and rank == 0) else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -611,6 +653,7 @@ def main():
             "baselines": baselines,
             "sweep": sweep,
             "decode": decode,
+            "user_cells": cells,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

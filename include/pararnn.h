@@ -218,6 +218,78 @@ PARARNN_API pararnn_status pararnn_lstm_adjoint(const void* u, pararnn_dtype u_d
                                     int64_t D, void* workspace, size_t workspace_bytes,
                                     pararnn_stream_t stream);
 
+/* ---------------------------------------------------- user-written cells */
+
+/* The fused solve for a cell the caller writes ("Como usar": the user writes
+ * only the recurrence step; Newton, the Jacobians and the parallel reduction
+ * are the library's).  `source` is CUDA C++ defining
+ *
+ *   template <class T>
+ *   __device__ void recurrence_step(const T* s, const float* u,
+ *                                   const float* a, T* out);
+ *
+ * for one (b, d) channel: s = its n_state components at step l-1, u = its
+ * n_gates gate pre-activations at step l, a = its n_gates recurrence
+ * weights, out = its n_state components at step l.  The body uses +, -, *,
+ * / and exp, log, tanh, sigmoid, sqrt, sin, cos (value_of(x) gives a plain
+ * float for branches); it runs with T = float for values and with a
+ * forward-mode dual number for the Jacobian block d out / d s, so the
+ * Jacobian is diagonal (n_state = 1) or one 2x2 block per channel
+ * (n_state = 2).  pararnn_cell_create compiles it with NVRTC into the same
+ * warp-specialised kernel as the built-in cells (dual-number Jacobians; the
+ * CUDA math library's expf/tanhf/..., or with PARARNN_CELL_FAST_MATH the
+ * hardware approximations), for sm_100a, and loads it on the current
+ * device.
+ *
+ * Returns PARARNN_ERR_INVALID_ARG if the source does not compile (the start
+ * of the compiler log is in pararnn_last_error(), all of it in
+ * pararnn_cell_compile_log()), PARARNN_ERR_UNSUPPORTED for n_gates outside
+ * 1..4, n_state outside 1..2 or when NVRTC cannot be loaded, and
+ * PARARNN_ERR_CUDA when the module cannot be loaded (no device, not sm_100).
+ * The handle belongs to the caller (pararnn_cell_destroy); it is bound to
+ * the device that was current at creation. */
+typedef struct pararnn_cell_st* pararnn_cell;
+
+/* flags of pararnn_cell_create */
+#define PARARNN_CELL_FAST_MATH 1u /* exp, log, tanh, sigmoid, sin, cos and the duals' divisions
+                                     from the hardware approximations (__expf, __fdividef, ...)
+                                     instead of the CUDA math library's accurate functions */
+
+PARARNN_API pararnn_status pararnn_cell_create(const char* source, int n_gates, int n_state,
+                                               unsigned flags, pararnn_cell* out);
+/* Compute warps per CTA (two steps each) of the kernel chosen for a gate
+ * dtype: the widest tile whose kernel spills at most 256 bytes a thread;
+ * 0 for a NULL cell. */
+PARARNN_API int pararnn_cell_compute_warps(pararnn_cell cell, pararnn_dtype u_dtype);
+PARARNN_API void pararnn_cell_destroy(pararnn_cell cell);
+/* Compiler log of the calling thread's last pararnn_cell_create ("" if none). */
+PARARNN_API const char* pararnn_cell_compile_log(void);
+/* Workspace bytes for one solve (0 = invalid shape); depends on u's dtype,
+ * which sets the tile. */
+PARARNN_API size_t pararnn_cell_workspace_size(pararnn_cell cell, pararnn_dtype u_dtype, int64_t B,
+                                               int64_t L, int64_t D);
+
+/* Newton solve of the cell's recurrence, with the stopping rule, outputs and
+ * errors of pararnn_gru_solve.
+ *   u   [B][L][n_gates][D] bf16 or fp32;  a [n_gates][D] fp32
+ *   s0  [n_state][B][D] fp32 initial state (NULL = zeros)
+ *   s   [n_state][B][L][D] fp32 out, components one after another
+ * Device pointers, 16-byte aligned; D a multiple of 8.  Synchronous like
+ * pararnn_gru_solve; the _async form returns after the launch and the
+ * outcome is read with pararnn_read_result. */
+PARARNN_API pararnn_status pararnn_cell_solve(pararnn_cell cell, const void* u, pararnn_dtype u_dtype,
+                                              const float* a, const float* s0, float* s, int64_t B,
+                                              int64_t L, int64_t D, float tol, int max_iters,
+                                              void* workspace, size_t workspace_bytes,
+                                              pararnn_stream_t stream, int* iters_out,
+                                              float* residual_out);
+PARARNN_API pararnn_status pararnn_cell_solve_async(pararnn_cell cell, const void* u,
+                                                    pararnn_dtype u_dtype, const float* a,
+                                                    const float* s0, float* s, int64_t B, int64_t L,
+                                                    int64_t D, float tol, int max_iters,
+                                                    void* workspace, size_t workspace_bytes,
+                                                    pararnn_stream_t stream);
+
 /* ----------------------------------------------------------- decode step */
 
 /* One recurrence step for B sequences at once, the token-by-token generation

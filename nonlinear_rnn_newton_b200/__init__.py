@@ -12,6 +12,13 @@ import importlib
 
 __all__ = [
     "PararnnError",
+    "pararnn_cell_compile_log",
+    "pararnn_cell_compute_warps",
+    "pararnn_cell_create",
+    "pararnn_cell_destroy",
+    "pararnn_cell_solve",
+    "pararnn_cell_solve_async",
+    "pararnn_cell_workspace_size",
     "pararnn_gru_adjoint",
     "pararnn_gru_adjoint_workspace_size",
     "pararnn_gru_sequential",

@@ -71,6 +71,16 @@ SIGNATURES = {
                                    _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "pararnn_gru_sequential": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "pararnn_lstm_sequential": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "pararnn_cell_create": (_st, [ctypes.c_char_p, ctypes.c_int, ctypes.c_int, ctypes.c_uint,
+                                  ctypes.POINTER(ctypes.c_void_p)]),
+    "pararnn_cell_compute_warps": (ctypes.c_int, [_vp, _st]),
+    "pararnn_cell_destroy": (None, [_vp]),
+    "pararnn_cell_compile_log": (ctypes.c_char_p, []),
+    "pararnn_cell_workspace_size": (ctypes.c_size_t, [_vp, _st, _i64, _i64, _i64]),
+    "pararnn_cell_solve": (_st, [_vp, _vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int, _vp,
+                                 ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float)]),
+    "pararnn_cell_solve_async": (_st, [_vp, _vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int,
+                                       _vp, ctypes.c_size_t, _vp]),
     "pararnn_gru_step": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _vp]),
     "pararnn_lstm_step": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp]),
     "pararnn_linear_scan": (_st, [_vp, _st, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
@@ -351,6 +361,76 @@ def pararnn_lstm_adjoint(u, a, c0, h0, c, h, dh, dc=None, du=None, da=None, dc0=
                                   _ptr(ws), ws.numel(), _stream(dev, stream))
     _check(st, allow=(OK,))
     return du, da, dc0, dh0
+
+
+# ------------------------------------------------------ user-written cells
+
+class CellHandle:
+    """A compiled user cell (owns the library handle; destroyed with the object)."""
+
+    def __init__(self, ptr, n_gates, n_state, log):
+        self.ptr, self.n_gates, self.n_state, self.log = ptr, n_gates, n_state, log
+
+    def __del__(self):
+        if getattr(self, "ptr", None) and lib is not None:
+            lib.pararnn_cell_destroy(self.ptr)
+            self.ptr = None
+
+
+CELL_FAST_MATH = 1
+
+
+def pararnn_cell_create(source, n_gates, n_state, flags=0):
+    """Compile `source` (which defines the templated recurrence_step) for the
+    current CUDA device; raises PararnnError with the compiler's log on error.
+    flags: CELL_FAST_MATH for the hardware approximations of the functions."""
+    h = ctypes.c_void_p()
+    st = lib.pararnn_cell_create(source.encode(), int(n_gates), int(n_state), int(flags), ctypes.byref(h))
+    _check(st, allow=(OK,))
+    return CellHandle(h, int(n_gates), int(n_state), pararnn_cell_compile_log())
+
+
+def pararnn_cell_destroy(cell):
+    if cell.ptr:
+        lib.pararnn_cell_destroy(cell.ptr)
+        cell.ptr = None
+
+
+def pararnn_cell_compute_warps(cell, u_dtype):
+    return int(lib.pararnn_cell_compute_warps(cell.ptr, BF16 if u_dtype == torch.bfloat16 else F32))
+
+
+def pararnn_cell_compile_log():
+    return lib.pararnn_cell_compile_log().decode()
+
+
+def pararnn_cell_workspace_size(cell, u_dtype, B, L, D):
+    code = BF16 if u_dtype == torch.bfloat16 else F32
+    return int(lib.pararnn_cell_workspace_size(cell.ptr, code, B, L, D))
+
+
+def pararnn_cell_solve(cell, u, a, s0=None, tol=1e-6, max_iters=10, s=None, workspace=None, stream=None):
+    """u [B, L, G, D]; a [G, D]; s0 [NS, B, D] or None -> (s [NS, B, L, D], iters, residual, status)."""
+    B, L, G, D = u.shape
+    s = s if s is not None else torch.empty((cell.n_state, B, L, D), dtype=torch.float32, device=u.device)
+    ws = _workspace(pararnn_cell_workspace_size(cell, u.dtype, B, L, D), u.device, workspace)
+    it, res = ctypes.c_int(0), ctypes.c_float(0.0)
+    with torch.cuda.device(u.device):
+        st = lib.pararnn_cell_solve(cell.ptr, _ptr(u), _dtype_code(u), _ptr(a), _ptr(s0), _ptr(s), B, L, D,
+                                    float(tol), int(max_iters), _ptr(ws), ws.numel(), _stream(u.device, stream),
+                                    ctypes.byref(it), ctypes.byref(res))
+    _check(st)
+    return s, it.value, res.value, st
+
+
+def pararnn_cell_solve_async(cell, u, a, s0, s, workspace, tol=1e-6, max_iters=10, stream=None):
+    B, L, G, D = u.shape
+    with torch.cuda.device(u.device):
+        st = lib.pararnn_cell_solve_async(cell.ptr, _ptr(u), _dtype_code(u), _ptr(a), _ptr(s0), _ptr(s), B, L, D,
+                                          float(tol), int(max_iters), _ptr(workspace), workspace.numel(),
+                                          _stream(u.device, stream))
+    _check(st, allow=(OK,))
+    return st
 
 
 # ------------------------------------------------------------- decode step

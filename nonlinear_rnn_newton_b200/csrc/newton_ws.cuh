@@ -101,7 +101,7 @@ struct NewtonWsLayout {
     static constexpr size_t smem_bytes = off_misc + misc_bytes;
     static constexpr int threads = 32 * (CW + 1);
     static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
-    static_assert(smem_bytes <= 232448, "shared memory");
+    static constexpr bool fits = smem_bytes <= 232448;  // opt-in shared memory per CTA
 };
 
 template <class Cell, class UT, int CW>
@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
     using Jac2 = typename Packed::Jac2;
     constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc;
     constexpr int kGroup = NS == 1 ? PARARNN_WS_GROUP_GRU : PARARNN_WS_GROUP_LSTM;
+    static_assert(LY::fits, "shared memory");
 
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + LY::off_misc);  // [kStages]

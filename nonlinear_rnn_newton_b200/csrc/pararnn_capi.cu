@@ -931,3 +931,6 @@ pararnn_status pararnn_selftest_wait_timeout(int which, int64_t limit_ns, void* 
 }
 
 }  // extern "C"
+
+// user-written cells, compiled at run time
+#include "cell_rtc_host.h"

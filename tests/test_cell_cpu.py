@@ -1,0 +1,66 @@
+"""The runtime-compiled cell path on the CPU: NVRTC compiles for sm_100a
+without a device, so source errors, argument checks and the generated
+kernels' resource use are checked here; loading the module needs a GPU."""
+import ctypes
+
+import pytest
+
+from tests.user_cells import CELLS
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from nonlinear_rnn_newton_b200 import build
+    build.build()
+    from nonlinear_rnn_newton_b200 import capi
+    return capi
+
+
+def create(capi, src, G, NS, flags=0):
+    h = ctypes.c_void_p()
+    st = capi.lib.pararnn_cell_create(src.encode() if src is not None else None, G, NS, flags, ctypes.byref(h))
+    return st, h
+
+
+def test_argument_checks(capi):
+    assert create(capi, None, 1, 1)[0] == capi.ERR_INVALID_ARG
+    assert capi.lib.pararnn_cell_create(b"x", 1, 1, 0, None) == capi.ERR_INVALID_ARG
+    assert create(capi, CELLS["elman"].source, 1, 1, flags=6)[0] == capi.ERR_INVALID_ARG
+    assert capi.lib.pararnn_cell_compute_warps(None, 1) == 0
+    assert create(capi, CELLS["elman"].source, 0, 1)[0] == capi.ERR_UNSUPPORTED
+    assert create(capi, CELLS["elman"].source, 5, 1)[0] == capi.ERR_UNSUPPORTED
+    assert create(capi, CELLS["elman"].source, 1, 3)[0] == capi.ERR_UNSUPPORTED
+    assert capi.lib.pararnn_cell_workspace_size(None, 1, 1, 64, 64) == 0
+    assert capi.lib.pararnn_cell_solve(None, 16, 1, 16, None, 16, 1, 8, 16, 1e-6, 10, 256, 1 << 20, None, None,
+                                       None) == capi.ERR_INVALID_ARG
+    capi.lib.pararnn_cell_destroy(None)  # no-op
+
+
+def test_source_errors_are_reported_with_the_log(capi):
+    bad = CELLS["elman"].source.replace("a[0] * s[0]", "a[0] * s_missing[0]")
+    st, h = create(capi, bad, 1, 1)
+    assert st == capi.ERR_INVALID_ARG and not h.value
+    assert "s_missing" in capi.last_error()
+    log = capi.lib.pararnn_cell_compile_log().decode()
+    assert "s_missing" in log and "recurrence_step" in log  # located in the user's source
+
+
+def test_a_step_without_the_template_signature_fails(capi):
+    st, _ = create(capi, "__device__ void recurrence_step(const float* s, const float* u, const float* a, "
+                         "float* out) { out[0] = s[0]; }", 1, 1)
+    assert st == capi.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+@pytest.mark.parametrize("name", sorted(CELLS))
+def test_cells_compile(capi, name, flags):
+    """Every test cell compiles, accurate and fast; without a GPU the module
+    load then fails."""
+    import torch
+    cell = CELLS[name]
+    st, h = create(capi, cell.source, cell.G, cell.NS, flags)
+    if torch.cuda.is_available():
+        assert st == capi.OK
+        capi.lib.pararnn_cell_destroy(h)
+    else:
+        assert st == capi.ERR_CUDA, capi.last_error()
