@@ -224,18 +224,18 @@ PARARNN_API pararnn_status pararnn_lstm_adjoint(const void* u, pararnn_dtype u_d
  * only the recurrence step; Newton, the Jacobians and the parallel reduction
  * are the library's).  `source` is CUDA C++ defining
  *
- *   template <class T>
- *   __device__ void recurrence_step(const T* s, const float* u,
- *                                   const float* a, T* out);
+ *   template <class T, class U>
+ *   __device__ void recurrence_step(const T* s, const U* u, const U* a,
+ *                                   T* out);
  *
  * for one (b, d) channel: s = its n_state components at step l-1, u = its
  * n_gates gate pre-activations at step l, a = its n_gates recurrence
  * weights, out = its n_state components at step l.  The body uses +, -, *,
  * / and exp, log, tanh, sigmoid, sqrt, sin, cos (value_of(x) gives a plain
- * float for branches); it runs with T = float for values and with a
- * forward-mode dual number for the Jacobian block d out / d s, so the
- * Jacobian is diagonal (n_state = 1) or one 2x2 block per channel
- * (n_state = 2).  pararnn_cell_create compiles it with NVRTC into the same
+ * float for branches).  It runs with T = U = float for values, with T a
+ * forward-mode dual number (U = float) for the Jacobian block d out / d s,
+ * and with T = U a dual number for the adjoint's derivatives; the Jacobian
+ * is diagonal (n_state = 1) or one 2x2 block per channel (n_state = 2).  pararnn_cell_create compiles it with NVRTC into the same
  * warp-specialised kernel as the built-in cells (dual-number Jacobians; the
  * CUDA math library's expf/tanhf/..., or with PARARNN_CELL_FAST_MATH the
  * hardware approximations), for sm_100a, and loads it on the current
@@ -283,6 +283,25 @@ PARARNN_API pararnn_status pararnn_cell_solve(pararnn_cell cell, const void* u, 
                                               void* workspace, size_t workspace_bytes,
                                               pararnn_stream_t stream, int* iters_out,
                                               float* residual_out);
+/* Training gradients through a user cell: the reverse-time adjoint of
+ * pararnn_gru_adjoint for the cell's own equations, at converged forward
+ * states s (from pararnn_cell_solve).  The derivatives of the step with
+ * respect to its state, gates and weights come from one forward-mode
+ * dual-number evaluation per step.
+ *   ds   [n_state][B][L][D] upstream gradient dLoss/ds, fp32, every component
+ *   du   [B][L][n_gates][D] fp32 out;  da [n_gates][D] fp32 out (overwritten)
+ *   ds0  [n_state][B][D] fp32 out, dLoss/ds0 (NULL = not wanted)
+ * Other arguments as for pararnn_cell_solve; the workspace comes from
+ * pararnn_cell_adjoint_workspace_size.  Asynchronous on `stream`; the
+ * status reports argument and launch errors. */
+PARARNN_API size_t pararnn_cell_adjoint_workspace_size(pararnn_cell cell, int64_t B, int64_t L,
+                                                       int64_t D);
+PARARNN_API pararnn_status pararnn_cell_adjoint(pararnn_cell cell, const void* u,
+                                                pararnn_dtype u_dtype, const float* a,
+                                                const float* s0, const float* s, const float* ds,
+                                                float* du, float* da, float* ds0, int64_t B,
+                                                int64_t L, int64_t D, void* workspace,
+                                                size_t workspace_bytes, pararnn_stream_t stream);
 PARARNN_API pararnn_status pararnn_cell_solve_async(pararnn_cell cell, const void* u,
                                                     pararnn_dtype u_dtype, const float* a,
                                                     const float* s0, float* s, int64_t B, int64_t L,

@@ -12,6 +12,8 @@ import importlib
 
 __all__ = [
     "PararnnError",
+    "pararnn_cell_adjoint",
+    "pararnn_cell_adjoint_workspace_size",
     "pararnn_cell_compile_log",
     "pararnn_cell_compute_warps",
     "pararnn_cell_create",

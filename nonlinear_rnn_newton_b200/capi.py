@@ -79,6 +79,9 @@ SIGNATURES = {
     "pararnn_cell_workspace_size": (ctypes.c_size_t, [_vp, _st, _i64, _i64, _i64]),
     "pararnn_cell_solve": (_st, [_vp, _vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int, _vp,
                                  ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float)]),
+    "pararnn_cell_adjoint_workspace_size": (ctypes.c_size_t, [_vp, _i64, _i64, _i64]),
+    "pararnn_cell_adjoint": (_st, [_vp, _vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                   ctypes.c_size_t, _vp]),
     "pararnn_cell_solve_async": (_st, [_vp, _vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int,
                                        _vp, ctypes.c_size_t, _vp]),
     "pararnn_gru_step": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _vp]),
@@ -421,6 +424,29 @@ def pararnn_cell_solve(cell, u, a, s0=None, tol=1e-6, max_iters=10, s=None, work
                                     ctypes.byref(it), ctypes.byref(res))
     _check(st)
     return s, it.value, res.value, st
+
+
+def pararnn_cell_adjoint_workspace_size(cell, B, L, D):
+    return int(lib.pararnn_cell_adjoint_workspace_size(cell.ptr, B, L, D))
+
+
+def pararnn_cell_adjoint(cell, u, a, s0, s, ds, du=None, da=None, ds0=None, want_ds0=True, workspace=None,
+                         stream=None):
+    """Gradients at converged states s [NS, B, L, D] for upstream ds [NS, B, L, D]
+    -> (du [B, L, G, D], da [G, D], ds0 [NS, B, D] or None)."""
+    B, L, G, D = u.shape
+    dev = u.device
+    du = du if du is not None else torch.empty((B, L, G, D), dtype=torch.float32, device=dev)
+    da = da if da is not None else torch.empty((G, D), dtype=torch.float32, device=dev)
+    if want_ds0 and ds0 is None:
+        ds0 = torch.empty((cell.n_state, B, D), dtype=torch.float32, device=dev)
+    ws = _workspace(pararnn_cell_adjoint_workspace_size(cell, B, L, D), dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib.pararnn_cell_adjoint(cell.ptr, _ptr(u), _dtype_code(u), _ptr(a), _ptr(s0), _ptr(s), _ptr(ds),
+                                      _ptr(du), _ptr(da), _ptr(ds0), B, L, D, _ptr(ws), ws.numel(),
+                                      _stream(dev, stream))
+    _check(st, allow=(OK,))
+    return du, da, ds0
 
 
 def pararnn_cell_solve_async(cell, u, a, s0, s, workspace, tol=1e-6, max_iters=10, stream=None):

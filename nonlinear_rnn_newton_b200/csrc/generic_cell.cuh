@@ -9,13 +9,19 @@
 //
 // Included after the user's source, which defines, inside namespace
 // pararnn_user,
-//     template <class T>
-//     __device__ void recurrence_step(const T* s, const float* u,
-//                                     const float* a, T* out);
+//     template <class T, class U>
+//     __device__ void recurrence_step(const T* s, const U* u, const U* a,
+//                                     T* out);
 // (s: the NS state components of one channel at step l-1; u: its G gate
 // pre-activations at step l; a: its G recurrence weights; out: the NS
-// components at step l).  The value comes from T = float; the Jacobian
-// block J[q][r] = d out_q / d s_r from one evaluation with T = Dual<NS>.
+// components at step l; T is the number type of the state, U that of the
+// inputs).  Three instantiations serve the solve and the adjoint:
+//   * value: T = U = float;
+//   * Jacobian block J[q][r] = d out_q / d s_r: T = Dual<NS>, U = float,
+//     the state components seeded with unit tangents;
+//   * vector-Jacobian products for the adjoint: T = U = Dual<NS + 2G>, with
+//     the state, the gates and the weights seeded, so that one evaluation
+//     gives d out / d (s, u, a) and lam^T times it.
 // The packed two-channel, two-row forms the solve kernel calls evaluate the
 // four (row, channel) pairs one after another.
 #pragma once
@@ -58,6 +64,16 @@ __device__ __forceinline__ void set_matrix_lane(Aff2<2>& m, int i, const float (
     }
 }
 
+__device__ __forceinline__ void set_matrix(Aff<1>& m, const float (&J)[1][1]) { m.m = J[0][0]; }
+
+__device__ __forceinline__ void set_matrix(Aff<2>& m, const float (&J)[2][2])
+{
+    m.m00 = J[0][0];
+    m.m01 = J[0][1];
+    m.m10 = J[1][0];
+    m.m11 = J[1][1];
+}
+
 __device__ __forceinline__ float lane_of(float2 x, int i) { return i == 0 ? x.x : x.y; }
 __device__ __forceinline__ void set_lane(float2& x, int i, float v)
 {
@@ -74,7 +90,7 @@ struct GenericCell {
 
     __device__ __forceinline__ static void value(const float* s, const float* u, const float* a, float* f)
     {
-        pararnn_user::recurrence_step<float>(s, u, a, f);
+        pararnn_user::recurrence_step<float, float>(s, u, a, f);
     }
 
     // f = step(s) and J[q][r] = d f_q / d s_r
@@ -87,12 +103,57 @@ struct GenericCell {
             x[q] = pararnn_user::Dual<NS>(s[q]);
             x[q].d[q] = 1.0f;
         }
-        pararnn_user::recurrence_step<pararnn_user::Dual<NS>>(x, u, a, y);
+        pararnn_user::recurrence_step<pararnn_user::Dual<NS>, float>(x, u, a, y);
 #pragma unroll
         for (int q = 0; q < NS; ++q) {
             f[q] = y[q].v;
 #pragma unroll
             for (int r = 0; r < NS; ++r) J[q][r] = y[q].d[r];
+        }
+    }
+
+    // f and its Jacobian in the matrix part of an affine map (the adjoint's form)
+    __device__ __forceinline__ static void eval(const float* s, const float* u, const float* a, float* f, Map& J)
+    {
+        float m[NS][NS];
+        value_jac(s, u, a, f, m);
+        set_matrix(J, m);
+    }
+
+    // Reverse mode at one step, lam = dLoss/d out: du_g = lam . d out/d u_g,
+    // dacc_g += lam . d out/d a_g, mu_r = lam . d out/d s_r.
+    __device__ __forceinline__ static void vjp(const float* s, const float* u, const float* a, const float* lam,
+                                               float* du, float* dacc, float* mu)
+    {
+        constexpr int K = NS + 2 * G;
+        using D = pararnn_user::Dual<K>;
+        D x[NS], uu[G], aa[G], y[NS];
+#pragma unroll
+        for (int q = 0; q < NS; ++q) {
+            x[q] = D(s[q]);
+            x[q].d[q] = 1.0f;
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            uu[g] = D(u[g]);
+            uu[g].d[NS + g] = 1.0f;
+            aa[g] = D(a[g]);
+            aa[g].d[NS + G + g] = 1.0f;
+        }
+        pararnn_user::recurrence_step<D, D>(x, uu, aa, y);
+        float t[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            t[k] = 0.0f;
+#pragma unroll
+            for (int q = 0; q < NS; ++q) t[k] = fmaf(lam[q], y[q].d[k], t[k]);
+        }
+#pragma unroll
+        for (int q = 0; q < NS; ++q) mu[q] = t[q];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            du[g] = t[NS + g];
+            dacc[g] += t[NS + G + g];
         }
     }
 

@@ -1,12 +1,13 @@
 """Example sources for pararnn_cell_create: the diagonal GRU and LSTM of the
 built-in solves, written as user cells (one recurrence step, templated on the
-number type; the library derives the Jacobians).  Gate order and equations
+number types of the state, T, and of the inputs, U; the library derives the
+Jacobians and the adjoint's derivatives).  Gate order and equations
 are those of the built-in cells: GRU (z, r, c) with the candidate on r*h,
 LSTM (i, f, o, g) over the state (c, h)."""
 
 GRU = r"""
-template <class T>
-__device__ void recurrence_step(const T* s, const float* u, const float* a, T* out)
+template <class T, class U>
+__device__ void recurrence_step(const T* s, const U* u, const U* a, T* out)
 {
     const T h = s[0];
     const T z = sigmoid(u[0] + a[0] * h);
@@ -17,8 +18,8 @@ __device__ void recurrence_step(const T* s, const float* u, const float* a, T* o
 """
 
 LSTM = r"""
-template <class T>
-__device__ void recurrence_step(const T* s, const float* u, const float* a, T* out)
+template <class T, class U>
+__device__ void recurrence_step(const T* s, const U* u, const U* a, T* out)
 {
     const T c = s[0], h = s[1];
     const T i = sigmoid(u[0] + a[0] * h);

@@ -67,6 +67,27 @@ def residual(step, ug, a, H, s0):
     return F
 
 
+def generic_bptt(step, u, a, s0, ds, ns):
+    """Gradients of Loss = sum over l of <ds_l, s_l> for the sequential states
+    s_l = step(s_{l-1}, u_l, a) (back-propagation through time), by torch
+    autograd in float64; `step` takes the array module as xp=torch.  ds
+    [NS, B, L, D].  Returns (du [B, L, G, D], da [G, D], ds0 [NS, B, D])."""
+    import torch
+    ug = torch.tensor(_gates(u), requires_grad=True)  # [L, G, B, D]
+    at = torch.tensor(_f64(a), requires_grad=True)
+    L, G, B, D = ug.shape
+    s0t = torch.zeros((ns, B, D), dtype=torch.float64) if s0 is None else torch.tensor(_f64(s0).reshape(ns, B, D))
+    s0t.requires_grad_(True)
+    dst = torch.tensor(_f64(ds))
+    s, loss = s0t, torch.zeros((), dtype=torch.float64)
+    for l in range(L):
+        s = step(s, ug[l], at, xp=torch)
+        loss = loss + (dst[:, :, l] * s).sum()
+    loss.backward()
+    du = ug.grad.permute(2, 0, 1, 3).numpy()
+    return du, at.grad.numpy(), s0t.grad.numpy()
+
+
 def generic_newton(step, jac, u, a, s0, ns, tol=1e-6, max_iters=10):
     """Serial Newton.  Returns (H [NS, B, L, D], iters, residual, status,
     residual history)."""

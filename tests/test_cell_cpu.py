@@ -49,6 +49,11 @@ def test_a_step_without_the_template_signature_fails(capi):
     st, _ = create(capi, "__device__ void recurrence_step(const float* s, const float* u, const float* a, "
                          "float* out) { out[0] = s[0]; }", 1, 1)
     assert st == capi.ERR_INVALID_ARG
+    # one number type for state and inputs is not enough either (the adjoint
+    # differentiates through u and a)
+    st, _ = create(capi, "template <class T> __device__ void recurrence_step(const T* s, const float* u, "
+                         "const float* a, T* out) { out[0] = s[0] * a[0] + u[0]; }", 1, 1)
+    assert st == capi.ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("flags", [0, 1])

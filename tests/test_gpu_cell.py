@@ -96,8 +96,8 @@ def test_tile_choice(cuda, compiled):
 def test_bad_source_on_gpu(cuda):
     from nonlinear_rnn_newton_b200 import capi
     with pytest.raises(capi.PararnnError) as e:
-        P().pararnn_cell_create("template <class T> __device__ void recurrence_step(const T* s, const float* u, "
-                                "const float* a, T* out) { out[0] = nothing; }", 1, 1)
+        P().pararnn_cell_create("template <class T, class U> __device__ void recurrence_step(const T* s, const U* u, "
+                                "const U* a, T* out) { out[0] = nothing; }", 1, 1)
     assert "nothing" in str(e.value)
 
 
@@ -116,3 +116,57 @@ def test_max_iters_and_tol_rules(cuda, compiled):
     s, it, r, st = P().pararnn_cell_solve(compiled["mixed", 0], ud, ad, sd, max_iters=1)
     H1, *_ = OG.generic_newton(cell.step, cell.jac, u, a, s0, 2, tol=0.0, max_iters=1)
     assert it == 1 and H.max_abs(s.cpu(), H1) <= TOL_STATE
+
+
+ADJ_SHAPES = [(2, 300, 136, "bf16"), (3, 257, 64, "f32"), (1, 1, 8, "bf16")]
+
+
+@pytest.mark.parametrize("fast", [0, 1])
+@pytest.mark.parametrize("name", sorted(CELLS))
+@pytest.mark.parametrize("B,L,D,dt", ADJ_SHAPES, ids=lambda v: str(v))
+def test_user_cell_adjoint_matches_bptt(cuda, compiled, name, B, L, D, dt, fast):
+    """Adjoint on the GPU solve's converged states against the oracle's BPTT
+    (torch autograd in float64 through its own sequential states).  du and
+    ds0 within 1e-4 * max(1, max|ref|); da within 1e-5 of sum_{b,l} |du| *
+    max|s| (every test cell takes its weights as a * (a state value) inside
+    a gate, so that bounds the sum of the absolute terms)."""
+    cell = CELLS[name]
+    u, a, s0 = draw(cell, B, L, D, dt, seed=3 * B + L)
+    ds = torch.randn((cell.NS, B, L, D), generator=torch.Generator().manual_seed(L))
+    ud, ad, sd = u.to(cuda), a.to(cuda), s0.to(cuda)
+    h = compiled[name, fast]
+    s, it, r, st = P().pararnn_cell_solve(h, ud, ad, sd, tol=1e-7, max_iters=20)
+    du, da, ds0 = P().pararnn_cell_adjoint(h, ud, ad, sd, s, ds.to(cuda))
+    torch.cuda.synchronize()
+    rdu, rda, rds0 = OG.generic_bptt(cell.step, u, a, s0, ds, cell.NS)
+    for x, ref in ((du, rdu), (ds0, rds0)):
+        scale = max(1.0, float(np.max(np.abs(ref))))
+        assert H.max_abs(x.cpu(), ref) <= 1e-4 * scale
+    smax = max(1.0, float(s.abs().max()))
+    bound = 1e-5 * np.sum(np.abs(rdu), axis=(0, 1)) * smax + 1e-6
+    assert np.all(np.abs(da.cpu().numpy() - rda) <= bound)
+
+
+def test_user_adjoints_match_the_builtin_ones(cuda, compiled):
+    """The GRU and LSTM written as user cells give the built-in adjoints'
+    gradients (to fp32 rounding of two different evaluation orders)."""
+    for name in ("gru", "lstm"):
+        cell = CELLS[name]
+        u, a, s0 = draw(cell, 2, 1024, 256, "bf16", seed=77)
+        ds = torch.randn((cell.NS, 2, 1024, 256), generator=torch.Generator().manual_seed(2)).to(cuda)
+        ud, ad, sd = u.to(cuda), a.to(cuda), s0.to(cuda)
+        s, *_ = P().pararnn_cell_solve(compiled[name, 0], ud, ad, sd, tol=1e-7, max_iters=20)
+        du, da, ds0 = P().pararnn_cell_adjoint(compiled[name, 0], ud, ad, sd, s, ds)
+        if name == "gru":
+            bdu, bda, bdh0 = P().pararnn_gru_adjoint(ud, ad, sd[0], s[0], ds[0])
+            bds0 = bdh0[None]
+        else:
+            bdu, bda, bdc0, bdh0 = P().pararnn_lstm_adjoint(ud, ad, sd[0], sd[1], s[0], s[1], ds[1], dc=ds[0])
+            bds0 = torch.stack([bdc0, bdh0])
+        torch.cuda.synchronize()
+        for x, ref in ((du, bdu), (ds0, bds0)):
+            scale = max(1.0, float(ref.abs().max()))
+            assert float((x - ref).abs().max()) <= 2e-5 * scale, name
+        smax = max(1.0, float(s.abs().max()))
+        bound = 1e-5 * bdu.abs().sum(dim=(0, 1)) * smax + 1e-6
+        assert bool(((da - bda).abs() <= bound).all()), name

@@ -110,3 +110,49 @@ def test_newton_converges_to_the_sequential_states(name):
     assert st == OG.OK and r <= 1e-10
     assert np.max(np.abs(H - OG.generic_seq(cell.step, u, a, s0, cell.NS))) < 1e-9
     assert all(np.diff(hist[-3:]) < 0)  # fast final decrease
+
+
+def test_bptt_matches_c_oracle_gru_and_lstm():
+    x = W.make_inputs(W.custom("gru", 2, 30, 16, "bf16", h0_std=0.1), seed=9)
+    g = torch.Generator().manual_seed(1)
+    dh = torch.randn((2, 30, 16), generator=g, dtype=torch.float64)
+    du, da, dh0 = oracle.gru_bptt(x.u, x.a, x.h0, dh)
+    gdu, gda, gds0 = OG.generic_bptt(CELLS["gru"].step, x.u, x.a, x.h0.double().numpy()[None], dh.numpy()[None], 1)
+    assert np.max(np.abs(gdu - du)) < 1e-12 and np.max(np.abs(gda - da)) < 1e-11
+    assert np.max(np.abs(gds0[0] - dh0)) < 1e-12
+    x = W.make_inputs(W.custom("lstm", 2, 25, 8, "f32", h0_std=0.1), seed=10)
+    dh = torch.randn((2, 25, 8), generator=g, dtype=torch.float64)
+    dc = torch.randn((2, 25, 8), generator=g, dtype=torch.float64)
+    du, da, dc0, dh0 = oracle.lstm_bptt(x.u, x.a, None, x.h0, dh, dc)
+    s0 = np.stack([np.zeros((2, 8)), x.h0.double().numpy()])
+    gdu, gda, gds0 = OG.generic_bptt(CELLS["lstm"].step, x.u, x.a, s0, np.stack([dc.numpy(), dh.numpy()]), 2)
+    assert np.max(np.abs(gdu - du)) < 1e-12 and np.max(np.abs(gda - da)) < 1e-11
+    assert np.max(np.abs(gds0[0] - dc0)) < 1e-12 and np.max(np.abs(gds0[1] - dh0)) < 1e-12
+
+
+@pytest.mark.parametrize("name", sorted(CELLS))
+def test_bptt_matches_finite_differences(name):
+    """d Loss / d u, d a, d s0 by central differences of the sequential
+    states, on a tiny problem, for a few sampled entries."""
+    cell = CELLS[name]
+    B, L, D = 1, 6, 2
+    u, a, s0 = inputs(cell, B, L, D, seed=17)
+    ds = np.random.default_rng(3).normal(size=(cell.NS, B, L, D))
+    du, da, ds0 = OG.generic_bptt(cell.step, u, a, s0, ds, cell.NS)
+    loss = lambda uu, aa, ss: float(np.sum(ds * OG.generic_seq(cell.step, uu, aa, ss, cell.NS)))
+    eps = 1e-6
+    for idx in [(0, 0, 0, 0), (0, L - 1, cell.G - 1, 1), (0, 2, 0, 1)]:
+        up, um = u.copy(), u.copy()
+        up[idx] += eps
+        um[idx] -= eps
+        assert abs((loss(up, a, s0) - loss(um, a, s0)) / (2 * eps) - du[idx]) < 1e-7
+    for idx in [(0, 0), (cell.G - 1, 1)]:
+        ap, am = a.copy(), a.copy()
+        ap[idx] += eps
+        am[idx] -= eps
+        assert abs((loss(u, ap, s0) - loss(u, am, s0)) / (2 * eps) - da[idx]) < 1e-7
+    for idx in [(0, 0, 0), (cell.NS - 1, 0, 1)]:
+        sp, sm = s0.copy(), s0.copy()
+        sp[idx] += eps
+        sm[idx] -= eps
+        assert abs((loss(u, a, sp) - loss(u, a, sm)) / (2 * eps) - ds0[idx]) < 1e-7

@@ -1,7 +1,8 @@
 """User-written cells for the tests of the runtime-compiled solve: each one is
 the CUDA source handed to pararnn_cell_create and, for the oracle, the same
-step and its Jacobian written in float64 numpy (vectorised over channels:
-s [NS, B, D], u [G, B, D], a [G, D])."""
+step and its Jacobian written in float64 (vectorised over channels:
+s [NS, B, D], u [G, B, D], a [G, D]).  The steps take the array module as
+`xp` (numpy, or torch for the autograd gradients of the oracle's BPTT)."""
 from dataclasses import dataclass
 from typing import Callable
 
@@ -10,8 +11,8 @@ import numpy as np
 from nonlinear_rnn_newton_b200 import example_cells
 
 
-def sig(x):
-    return 1.0 / (1.0 + np.exp(-x))
+def sig(x, xp=np):
+    return 1.0 / (1.0 + xp.exp(-x))
 
 
 @dataclass
@@ -29,11 +30,11 @@ class UserCell:
 GRU_SRC = example_cells.GRU
 
 
-def gru_step(s, u, a):
+def gru_step(s, u, a, xp=np):
     h = s[0]
-    z = sig(u[0] + a[0] * h)
-    r = sig(u[1] + a[1] * h)
-    c = np.tanh(u[2] + a[2] * r * h)
+    z = sig(u[0] + a[0] * h, xp)
+    r = sig(u[1] + a[1] * h, xp)
+    c = xp.tanh(u[2] + a[2] * r * h)
     return ((1 - z) * h + z * c)[None]
 
 
@@ -51,12 +52,12 @@ def gru_jac(s, u, a):
 LSTM_SRC = example_cells.LSTM
 
 
-def lstm_step(s, u, a):
-    c, h = s
-    i, f, o = sig(u[0] + a[0] * h), sig(u[1] + a[1] * h), sig(u[2] + a[2] * h)
-    g = np.tanh(u[3] + a[3] * h)
+def lstm_step(s, u, a, xp=np):
+    c, h = s[0], s[1]
+    i, f, o = sig(u[0] + a[0] * h, xp), sig(u[1] + a[1] * h, xp), sig(u[2] + a[2] * h, xp)
+    g = xp.tanh(u[3] + a[3] * h)
     cn = f * c + i * g
-    return np.stack([cn, o * np.tanh(cn)])
+    return xp.stack([cn, o * xp.tanh(cn)])
 
 
 def lstm_jac(s, u, a):
@@ -76,16 +77,16 @@ def lstm_jac(s, u, a):
 # -------------------------------------------------- diagonal Elman (tanh)
 
 ELMAN_SRC = r"""
-template <class T>
-__device__ void recurrence_step(const T* s, const float* u, const float* a, T* out)
+template <class T, class U>
+__device__ void recurrence_step(const T* s, const U* u, const U* a, T* out)
 {
     out[0] = tanh(u[0] + a[0] * s[0]);
 }
 """
 
 
-def elman_step(s, u, a):
-    return np.tanh(u[0] + a[0] * s[0])[None]
+def elman_step(s, u, a, xp=np):
+    return xp.tanh(u[0] + a[0] * s[0])[None]
 
 
 def elman_jac(s, u, a):
@@ -98,8 +99,8 @@ def elman_jac(s, u, a):
 MIXED_SRC = r"""
 // x, y coupled both ways; uses +, -, *, /, sin, cos, sqrt, exp, log,
 // sigmoid and tanh on duals
-template <class T>
-__device__ void recurrence_step(const T* s, const float* u, const float* a, T* out)
+template <class T, class U>
+__device__ void recurrence_step(const T* s, const U* u, const U* a, T* out)
 {
     const T x = s[0], y = s[1];
     const T p = u[0] + a[0] * y;
@@ -111,13 +112,13 @@ __device__ void recurrence_step(const T* s, const float* u, const float* a, T* o
 """
 
 
-def mixed_step(s, u, a):
-    x, y = s
+def mixed_step(s, u, a, xp=np):
+    x, y = s[0], s[1]
     p = u[0] + a[0] * y
     q = u[1] + a[1] * x
-    o0 = 0.5 * np.sin(p) + 0.5 * x / np.sqrt(1 + x * x)
-    o1 = sig(q) * np.tanh(y) + 0.2 * np.log(1 + np.exp(-q * q)) / (1.25 + np.cos(y))
-    return np.stack([o0, o1])
+    o0 = 0.5 * xp.sin(p) + 0.5 * x / xp.sqrt(1 + x * x)
+    o1 = sig(q, xp) * xp.tanh(y) + 0.2 * xp.log(1 + xp.exp(-q * q)) / (1.25 + xp.cos(y))
+    return xp.stack([o0, o1])
 
 
 def mixed_jac(s, u, a):
