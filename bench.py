@@ -62,6 +62,21 @@ def solve_bytes(w: W.Workload, iters: int) -> int:
     return w.N * (first + (max(iters, 1) - 1) * later)
 
 
+def pass_bytes(w: W.Workload, k: int) -> int:
+    """Bytes Newton pass k must move (pass 0 starts from the zero guess and
+    reads no states)."""
+    es = 2 if w.u_dtype == "bf16" else 4
+    ns = 1 if w.cell == "gru" else 2
+    return w.N * (w.G * es + (1 if k == 0 else 2) * ns * 4)
+
+
+def per_pass(w: W.Workload, pass_us, peak):
+    """Per-iteration roofline from the solve's device pass timestamps."""
+    return [{"pass": k, "us": round(us, 2), "bytes": pass_bytes(w, k),
+             "gbs": pass_bytes(w, k) / (us * 1e-6) / 1e9, "frac": pass_bytes(w, k) / (us * 1e-6) / 1e9 / peak}
+            for k, us in enumerate(pass_us) if us > 0]
+
+
 def adjoint_bytes(w: W.Workload) -> int:
     """The adjoint reads gates, forward states (and the state before each
     step, which is the previous row of the same arrays) and the upstream
@@ -243,6 +258,9 @@ class Step:
 
     def result(self):
         return self.P.pararnn_read_result(self.ws, self.stream)
+
+    def pass_times(self):
+        return self.P.pararnn_read_pass_times(self.ws, self.stream)
 
 
 def events(n, k):
@@ -602,7 +620,8 @@ def main():
     kname = "newton_solve_ws_kernel"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": profile_traffic(kname, w.name), "peak_kind": peak_kind, "kernel": kname,
-                "algorithmic_bytes_per_launch": algo, "kernel_ms_mean": solve_ms}
+                "algorithmic_bytes_per_launch": algo, "kernel_ms_mean": solve_ms,
+                "per_pass": per_pass(w, step.pass_times(), peak)}
     adjoint = None
     if w.train:
         ab = adjoint_bytes(w)

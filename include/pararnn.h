@@ -309,6 +309,16 @@ PARARNN_API pararnn_status pararnn_cell_solve_async(pararnn_cell cell, const voi
                                                     void* workspace, size_t workspace_bytes,
                                                     pararnn_stream_t stream);
 
+/* Duration of each Newton pass of the last solve run on `workspace` (the
+ * built-in and user-cell solves), from device timestamps the kernel takes
+ * when every CTA has finished a pass: pass_us[i] = microseconds of pass i,
+ * pass 0 from the kernel's start; *n_passes = passes recorded (at most 15).
+ * Synchronises `stream`.  The durations include the grid barrier that ends
+ * each pass; they sum to the kernel's time less its prologue and epilogue.
+ * The per-iteration roofline is (bytes a pass moves) / pass_us[i]. */
+PARARNN_API pararnn_status pararnn_read_pass_times(const void* workspace, pararnn_stream_t stream,
+                                                   double* pass_us, int max_passes, int* n_passes);
+
 /* ----------------------------------------------------------- decode step */
 
 /* One recurrence step for B sequences at once, the token-by-token generation

@@ -39,6 +39,7 @@ __all__ = [
     "pararnn_lstm_solve_async",
     "pararnn_lstm_step",
     "pararnn_lstm_workspace_size",
+    "pararnn_read_pass_times",
     "pararnn_read_result",
     "pararnn_selftest_wait_timeout",
 ]

@@ -65,6 +65,8 @@ SIGNATURES = {
     "pararnn_lstm_solve_async": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                        ctypes.c_float, ctypes.c_int, _vp, ctypes.c_size_t, _vp]),
     "pararnn_read_result": (_st, [_vp, _vp, ctypes.POINTER(Result)]),
+    "pararnn_read_pass_times": (_st, [_vp, _vp, ctypes.POINTER(ctypes.c_double), ctypes.c_int,
+                                      ctypes.POINTER(ctypes.c_int)]),
     "pararnn_gru_adjoint": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                   ctypes.c_size_t, _vp]),
     "pararnn_lstm_adjoint": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -320,6 +322,15 @@ def pararnn_read_result(workspace, stream=None):
     if st in (ERR_INVALID_ARG, ERR_WORKSPACE, ERR_CUDA):
         raise PararnnError(st, last_error())
     return r.status, r.iters, r.residual, r.residual0
+
+
+def pararnn_read_pass_times(workspace, stream=None):
+    """Synchronise and return the last solve's per-pass durations (us)."""
+    buf = (ctypes.c_double * 16)()
+    n = ctypes.c_int(0)
+    st = lib.pararnn_read_pass_times(_ptr(workspace), _stream(workspace.device, stream), buf, 16, ctypes.byref(n))
+    _check(st, allow=(OK,))
+    return [buf[i] for i in range(n.value)]
 
 
 # ---------------------------------------------------------------- adjoints

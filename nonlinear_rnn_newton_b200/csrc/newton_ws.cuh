@@ -149,6 +149,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
         prefetch_tensormap(&tm_bnd);
     }
 
+    if (tid == 0 && blockIdx.x == 0) hdr->t_pass[0] = global_timer_ns();
+
     for (int k = 0;; ++k) {
         const int slot = k % 3;
         const bool first = (k == 0);
@@ -669,6 +671,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 
         const bool bar_ok = grid_barrier(&hdr->bar, unsigned(k), err, p.wait_ns, &s_int[1]);
         if (tid == 0) {
+            // every CTA has finished pass k
+            if (blockIdx.x == 0 && k + 1 < kPassTimes) hdr->t_pass[k + 1] = global_timer_ns();
             NewtonDecision d = newton_decide(hdr, k, slot, bar_ok, p.tol, p.max_iters);
             if (!d.cont && blockIdx.x == 0) newton_publish(hdr, d, k);
             s_int[2] = d.cont;

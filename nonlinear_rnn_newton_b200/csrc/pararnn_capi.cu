@@ -760,6 +760,21 @@ pararnn_status pararnn_lstm_solve(const void* u, pararnn_dtype u_dtype, const fl
     return finish_sync(workspace, reinterpret_cast<cudaStream_t>(stream), iters_out, residual_out);
 }
 
+pararnn_status pararnn_read_pass_times(const void* workspace, pararnn_stream_t stream, double* pass_us, int max_passes,
+                                       int* n_passes)
+{
+    t_err[0] = '\0';
+    if (max_passes < 0 || (max_passes > 0 && !pass_us)) return fail(PARARNN_ERR_INVALID_ARG, "pass_us is NULL");
+    WsHeader h;
+    TRY(read_header(workspace, reinterpret_cast<cudaStream_t>(stream), &h));
+    int n = 0;
+    while (n + 1 < kPassTimes && h.t_pass[n + 1] != 0 && h.t_pass[n + 1] >= h.t_pass[n]) ++n;
+    if (h.t_pass[0] == 0) n = 0;
+    for (int i = 0; i < n && i < max_passes; ++i) pass_us[i] = double(h.t_pass[i + 1] - h.t_pass[i]) * 1e-3;
+    if (n_passes) *n_passes = n;
+    return PARARNN_OK;
+}
+
 pararnn_status pararnn_read_result(const void* workspace, pararnn_stream_t stream, pararnn_result* result)
 {
     WsHeader h;

@@ -26,6 +26,10 @@ constexpr int kDc = 32 * kV;       // channels per tile (one per lane x kV)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // First 256 bytes of every workspace.  Zeroed by the host before each run.
+// Pass boundaries the fused solve timestamps (%globaltimer, ns): the start of
+// pass 0 and the end of each of the first kPassTimes - 1 passes.
+constexpr int kPassTimes = 16;
+
 struct alignas(256) WsHeader {
     unsigned tick[4];  // tile ticket counter per pass slot (pass k uses k % 3)
     unsigned res[4];   // max |F| bits of the updated states per pass slot
@@ -34,7 +38,8 @@ struct alignas(256) WsHeader {
     int error;         // first device-side error (pararnn_status < 0), 0 if none
     int passes;        // Newton passes run
     pararnn_result result;
-    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result)];
+    unsigned long long t_pass[kPassTimes];  // see kPassTimes (0 = not reached)
+    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result) - 8 * kPassTimes];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
 

@@ -99,6 +99,9 @@ def test_argument_checks_before_any_gpu_work(capi):
     assert lib.pararnn_gru_sequential(16, 1, None, None, 16, 1, 8, 16, None) == E.ERR_INVALID_ARG
     assert lib.pararnn_linear_scan(16, 1, None, 16, 1, 8, 16, 256, 10, None) == E.ERR_WORKSPACE
     assert lib.pararnn_selftest_wait_timeout(5, 10, 256, 16384, None) == E.ERR_INVALID_ARG
+    n = ctypes.c_int(0)
+    assert lib.pararnn_read_pass_times(None, None, None, 0, ctypes.byref(n)) == E.ERR_WORKSPACE
+    assert lib.pararnn_read_pass_times(256, None, None, 4, ctypes.byref(n)) == E.ERR_INVALID_ARG
 
 
 def test_decode_step_checks(capi):

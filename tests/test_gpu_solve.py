@@ -188,6 +188,30 @@ def test_solve_is_deterministic(cuda):
     assert i1 == i2 and r1 == r2 and torch.equal(h1, h2)
 
 
+def test_pass_times(cuda):
+    """One timestamp per finished pass: as many passes as updates (one when
+    the initial guess already satisfies the rule), each positive, summing to
+    most of the launch's CUDA-event time."""
+    pk = P()
+    w = W.custom("gru", 4, 4096, 512, "bf16", h0_std=0.1)
+    x = W.make_inputs(w, seed=17).to(cuda)
+    h = torch.empty((w.B, w.L, w.D), device=cuda)
+    ws = torch.empty(pk.pararnn_gru_workspace_size(w.B, w.L, w.D), dtype=torch.uint8, device=cuda)
+    s = torch.cuda.current_stream()
+    for tol, max_iters in ((1e-6, 10), (1e30, 10), (0.0, 3)):
+        pk.pararnn_gru_solve_async(x.u, x.a, x.h0, h, ws, tol, max_iters)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        pk.pararnn_gru_solve_async(x.u, x.a, x.h0, h, ws, tol, max_iters)
+        e1.record(s)
+        st, it, r, r0 = pk.pararnn_read_result(ws)
+        us = pk.pararnn_read_pass_times(ws)
+        assert len(us) == max(it, 1), (tol, max_iters, it, us)
+        assert all(t > 0 for t in us)
+        total = e0.elapsed_time(e1) * 1e3
+        assert 0.3 * total <= sum(us) <= 1.02 * total, (us, total)
+
+
 def test_sequential_baselines_match_oracle(cuda):
     w = W.custom("gru", 3, 500, 136, "bf16", h0_std=0.1)
     x = W.make_inputs(w, seed=15)
