@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-cpu-baseline] [--sweep] [--decode] [--cells]
+                    [--seq-segments R1,R2,...]
 
 A step is one pass of the whole hot path over the workload through the C ABI:
 one full Newton solve (every iteration until convergence, the convergence
@@ -408,6 +409,36 @@ def run_cells(dev, stream, reps=5):
     return out
 
 
+def run_segments(w, xd, dev, stream, counts, reps=3):
+    """The solve with each sequence split into R segments (the multi-GPU
+    sequence sharding), all R run one after another on this GPU: time per
+    solve and iterations, beside the unsplit solve."""
+    from nonlinear_rnn_newton_b200 import sharded as SH
+    ns = 1 if w.cell == "gru" else 2
+    s0 = torch.zeros((ns, w.B, w.D), device=dev)
+    if xd.h0 is not None:
+        s0[ns - 1] = xd.h0
+    out = []
+    for R in counts:
+        edges = [round(i * w.L / R) for i in range(R + 1)]
+        segs = [SH.Segment(w.cell, xd.u[:, edges[r]:edges[r + 1]].contiguous(), xd.a, r, stream=stream)
+                for r in range(R)]
+        run = lambda: SH.solve_segments(segs, SH.LocalComm(), s0, w.tol, w.max_iters)
+        run()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            it, r, st = run()
+        e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        out.append({"segments": R, "ms": round(ms, 3), "ms_per_segment": round(ms / R, 3), "iters": it,
+                    "status": st, "residual": r})
+        del segs
+        torch.cuda.empty_cache()
+    return out
+
+
 def oracle_sample(w, x, rows, chans):
     """Sub-problem of the workload the oracle is timed on: the first `rows`
     batch rows and `chans` channels (channels are independent, so this is the
@@ -563,6 +594,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep (B=1, D=2048)")
     ap.add_argument("--decode", action="store_true", help="add the decode-step timings (CUDA graph of steps)")
     ap.add_argument("--cells", action="store_true", help="add the runtime-compiled user cells (GRU, LSTM sources)")
+    ap.add_argument("--seq-segments", default="", help="comma list of R: the solve with each sequence split into "
+                    "R segments (sequence sharding), run on this GPU one segment after another")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.BY_NAME[args.workload]
@@ -643,6 +676,9 @@ def main():
     sweep = run_sweep(dev, stream) if (args.sweep and rank == 0) else None
     decode = run_decode(dev, stream) if (args.decode and rank == 0) else None
     cells = run_cells(dev, stream) if (args.cells and rank == 0) else None
+    segments = None
+    if args.seq_segments and rank == 0:
+        segments = run_segments(w, xd, dev, stream, [int(v) for v in args.seq_segments.split(",")])
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -673,6 +709,7 @@ def main():
             "sweep": sweep,
             "decode": decode,
             "user_cells": cells,
+            "seq_segments": segments,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -319,6 +319,69 @@ PARARNN_API pararnn_status pararnn_cell_solve_async(pararnn_cell cell, const voi
 PARARNN_API pararnn_status pararnn_read_pass_times(const void* workspace, pararnn_stream_t stream,
                                                    double* pass_us, int max_passes, int* n_passes);
 
+/* ------------------------------------------------- segments of a sequence */
+
+/* The Newton solve with the sequence split into segments, one per GPU ("A
+ * sacada: método de Newton": every iteration solves a linear recurrence;
+ * over a segment its solution is affine in the state entering the
+ * segment).  One iteration k -> k+1 on each segment:
+ *   1. pararnn_*_segment_pass with s_carry = 0 (beta), then once per state
+ *      component j with s_carry = e_j (unit j), each from the same iterate;
+ *   2. gather the passes' last-step states of every segment, in segment
+ *      order, into ends [R][1 + NS][NS][B][D] (the exchange between GPUs);
+ *   3. pararnn_segment_carries -> the state entering every segment;
+ *   4. pararnn_*_segment_update with this segment's carry -> the iterate
+ *      k+1 and its residual; the maximum over segments decides.
+ * The iterate entering a segment at k+1 is its carry, which is also the
+ * state the next pass linearises the segment's first step at.
+ * Components are stacked one after another: [NS][B][Ls][D] for states over
+ * the segment, [NS][B][D] for one step (LSTM: c, then h).  Device pointers,
+ * 16-byte aligned, D a multiple of 8; all calls asynchronous on `stream`.
+ *
+ * segment_pass: one pass over the segment (gates u [B][Ls][G][D] of its
+ * steps) from the iterate s_in (NULL = the zero guess H^0), linearising the
+ * first step at s_lin (the iterate's state before the segment; NULL = 0),
+ * with s_carry (NULL = 0) as the new state before it.  Writes s_out (must not
+ * overlap s_in) and, if s_end is not NULL, the last step's states.  The
+ * workspace is the solve's (pararnn_*_workspace_size(B, Ls, D)). */
+PARARNN_API pararnn_status pararnn_gru_segment_pass(const void* u, pararnn_dtype u_dtype,
+                                                    const float* a, const float* h_in,
+                                                    const float* h_lin, const float* h_carry,
+                                                    float* h_out, float* h_end, int64_t B,
+                                                    int64_t L, int64_t D, void* workspace,
+                                                    size_t workspace_bytes,
+                                                    pararnn_stream_t stream);
+PARARNN_API pararnn_status pararnn_lstm_segment_pass(const void* u, pararnn_dtype u_dtype,
+                                                     const float* a, const float* s_in,
+                                                     const float* s_lin, const float* s_carry,
+                                                     float* s_out, float* s_end, int64_t B,
+                                                     int64_t L, int64_t D, void* workspace,
+                                                     size_t workspace_bytes,
+                                                     pararnn_stream_t stream);
+/* segment_update: s_out = beta + sum_j (unit_j - beta) carry_j, with beta
+ * [NS][B][Ls][D], unit [NS][NS][B][Ls][D] (pass j, then component), carry
+ * [NS][B][D]; and max |s_l - f(s_{l-1}, u_l)| over the segment (s_{-1} =
+ * carry) combined into *residual, a device float the caller sets to 0 first
+ * (a maximum over launches; NaN kept). */
+PARARNN_API pararnn_status pararnn_gru_segment_update(const void* u, pararnn_dtype u_dtype,
+                                                      const float* a, const float* beta,
+                                                      const float* unit, const float* carry,
+                                                      float* h_out, float* residual, int64_t B,
+                                                      int64_t L, int64_t D,
+                                                      pararnn_stream_t stream);
+PARARNN_API pararnn_status pararnn_lstm_segment_update(const void* u, pararnn_dtype u_dtype,
+                                                       const float* a, const float* beta,
+                                                       const float* unit, const float* carry,
+                                                       float* s_out, float* residual, int64_t B,
+                                                       int64_t L, int64_t D,
+                                                       pararnn_stream_t stream);
+/* segment_carries: from ends [R][1 + NS][NS][B][D] and the initial state s0
+ * [NS][B][D] (NULL = 0), the state entering every segment, carries
+ * [R][NS][B][D]: c_0 = s0, c_{r+1} = beta_r + sum_j (unit_rj - beta_r) c_r[j]. */
+PARARNN_API pararnn_status pararnn_segment_carries(const float* ends, const float* s0,
+                                                   float* carries, int n_segments, int n_state,
+                                                   int64_t B, int64_t D, pararnn_stream_t stream);
+
 /* ----------------------------------------------------------- decode step */
 
 /* One recurrence step for B sequences at once, the token-by-token generation

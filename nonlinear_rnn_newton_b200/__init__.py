@@ -23,6 +23,8 @@ __all__ = [
     "pararnn_cell_workspace_size",
     "pararnn_gru_adjoint",
     "pararnn_gru_adjoint_workspace_size",
+    "pararnn_gru_segment_pass",
+    "pararnn_gru_segment_update",
     "pararnn_gru_sequential",
     "pararnn_gru_solve",
     "pararnn_gru_solve_async",
@@ -34,12 +36,15 @@ __all__ = [
     "pararnn_linear_scan_workspace_size",
     "pararnn_lstm_adjoint",
     "pararnn_lstm_adjoint_workspace_size",
+    "pararnn_lstm_segment_pass",
+    "pararnn_lstm_segment_update",
     "pararnn_lstm_sequential",
     "pararnn_lstm_solve",
     "pararnn_lstm_solve_async",
     "pararnn_lstm_step",
     "pararnn_lstm_workspace_size",
     "pararnn_read_pass_times",
+    "pararnn_segment_carries",
     "pararnn_read_result",
     "pararnn_selftest_wait_timeout",
 ]

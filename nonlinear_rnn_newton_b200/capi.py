@@ -86,6 +86,13 @@ SIGNATURES = {
                                    ctypes.c_size_t, _vp]),
     "pararnn_cell_solve_async": (_st, [_vp, _vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, ctypes.c_int,
                                        _vp, ctypes.c_size_t, _vp]),
+    "pararnn_gru_segment_pass": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                       ctypes.c_size_t, _vp]),
+    "pararnn_lstm_segment_pass": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                        ctypes.c_size_t, _vp]),
+    "pararnn_gru_segment_update": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "pararnn_lstm_segment_update": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "pararnn_segment_carries": (_st, [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _i64, _i64, _vp]),
     "pararnn_gru_step": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _vp]),
     "pararnn_lstm_step": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp]),
     "pararnn_linear_scan": (_st, [_vp, _st, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
@@ -468,6 +475,47 @@ def pararnn_cell_solve_async(cell, u, a, s0, s, workspace, tol=1e-6, max_iters=1
                                           _stream(u.device, stream))
     _check(st, allow=(OK,))
     return st
+
+
+# ------------------------------------------------- segments of a sequence
+
+def _segment_pass(fn, u, a, s_in, s_lin, s_carry, s_out, s_end, workspace, stream):
+    B, L, G, D = u.shape
+    st = fn(_ptr(u), _dtype_code(u), _ptr(a), _ptr(s_in), _ptr(s_lin), _ptr(s_carry), _ptr(s_out), _ptr(s_end),
+            B, L, D, _ptr(workspace), workspace.numel(), _stream(u.device, stream))
+    _check(st, allow=(OK,))
+
+
+def pararnn_gru_segment_pass(u, a, h_in, h_lin, h_carry, h_out, h_end=None, workspace=None, stream=None):
+    """One Newton pass over a segment; states [1, B, Ls, D] / [1, B, D] (None = zeros)."""
+    _segment_pass(lib.pararnn_gru_segment_pass, u, a, h_in, h_lin, h_carry, h_out, h_end, workspace, stream)
+
+
+def pararnn_lstm_segment_pass(u, a, s_in, s_lin, s_carry, s_out, s_end=None, workspace=None, stream=None):
+    """One Newton pass over a segment; states [2, B, Ls, D] / [2, B, D] (c, h; None = zeros)."""
+    _segment_pass(lib.pararnn_lstm_segment_pass, u, a, s_in, s_lin, s_carry, s_out, s_end, workspace, stream)
+
+
+def _segment_update(fn, u, a, beta, unit, carry, s_out, residual, stream):
+    B, L, G, D = u.shape
+    st = fn(_ptr(u), _dtype_code(u), _ptr(a), _ptr(beta), _ptr(unit), _ptr(carry), _ptr(s_out), _ptr(residual),
+            B, L, D, _stream(u.device, stream))
+    _check(st, allow=(OK,))
+
+
+def pararnn_gru_segment_update(u, a, beta, unit, carry, h_out, residual, stream=None):
+    _segment_update(lib.pararnn_gru_segment_update, u, a, beta, unit, carry, h_out, residual, stream)
+
+
+def pararnn_lstm_segment_update(u, a, beta, unit, carry, s_out, residual, stream=None):
+    _segment_update(lib.pararnn_lstm_segment_update, u, a, beta, unit, carry, s_out, residual, stream)
+
+
+def pararnn_segment_carries(ends, s0, carries, stream=None):
+    """ends [R, 1 + NS, NS, B, D], s0 [NS, B, D] or None -> carries [R, NS, B, D]."""
+    R, _, NS, B, D = ends.shape
+    st = lib.pararnn_segment_carries(_ptr(ends), _ptr(s0), _ptr(carries), R, NS, B, D, _stream(ends.device, stream))
+    _check(st, allow=(OK,))
 
 
 # ------------------------------------------------------------- decode step

@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 
     for (int k = 0;; ++k) {
         const int slot = k % 3;
-        const bool first = (k == 0);
+        const bool first = (k == 0) && !p.warm;  // the pass starts from H^0 = 0
         if (tid == 0) {
             if (blockIdx.x == 0) {
                 // slot (k+1)%3 was last used two passes ago; every CTA is past it
@@ -425,7 +425,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                         F4 x{{0.f, 0.f, 0.f, 0.f}};
                         if (w == 0) {
                             if (c == 0) {
-                                if (chv && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+                                const float* lin = p.slin[q] ? p.slin[q] : p.s0[q];
+                                if (chv && lin) x = load4(lin + b * D + dch);
                             } else if (!first) {
                                 x = load4(sbnd + q * kDc + lane * kV);
                             }

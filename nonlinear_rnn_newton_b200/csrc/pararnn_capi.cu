@@ -21,6 +21,7 @@
 #include "newton_ws.cuh"
 #include "sequential.cuh"
 #include "decode.cuh"
+#include "segment.cuh"
 #include "adjoint.cuh"
 #include "linear_scan.cuh"
 
@@ -283,9 +284,12 @@ pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid, int th
 
 // ----------------------------------------------------------------- solves
 
+// in: where the first pass reads the states (segment passes: the given
+// iterate; NULL = st); slin, warm: see NewtonParams.
 template <class Cell, class UT, int T>
 pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
-                             float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream)
+                             float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream,
+                             const float* const* in = nullptr, const float* const* slin = nullptr, int warm = 0)
 {
     constexpr int NS = Cell::NS;
     constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
@@ -306,10 +310,11 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
 
     CUtensorMap tu, t0, t1;
     TRY(map_gates(&tu, u, dt, Cell::G, Cell::G, s, KL::Lc));
-    TRY(map_state(&t0, st[0], s, KL::Lc));
-    TRY(map_state(&t1, st[NS - 1], s, KL::Lc));
+    const float* src[2] = {in ? in[0] : st[0], in ? in[NS - 1] : st[NS - 1]};
+    TRY(map_state(&t0, src[0], s, KL::Lc));
+    TRY(map_state(&t1, src[1], s, KL::Lc));
 
-    NewtonParams p;
+    NewtonParams p{};
     p.a = a;
     p.s0[0] = s0[0];
     p.s0[1] = s0[1];
@@ -327,6 +332,16 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
     p.desc = reinterpret_cast<unsigned long long*>(wsb + ly.desc);
     p.bnd = reinterpret_cast<float*>(wsb + ly.extra);
     p.wait_ns = kWaitLimitNs;
+    p.slin[0] = slin ? slin[0] : nullptr;
+    p.slin[1] = slin ? slin[1] : nullptr;
+    p.warm = warm;
+    if (warm && s.n_chunks > 1) {
+        const long long n = (long long)NS * s.B * (s.n_chunks - 1) * (s.D / 4);
+        bnd_gather_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(src[0], src[1], p.bnd, NS, s.B, s.L, s.D,
+                                                                          s.n_chunks, KL::Lc, s.S * kDc);
+        CUDA_TRY(cudaGetLastError());
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
 
     int grid = 0;
     TRY(resident_grid(kern, KL::smem_bytes, s.n_tiles, &grid, threads));
@@ -394,6 +409,111 @@ pararnn_status solve_async(int cell, const void* u, pararnn_dtype dt, const floa
     }
     TRY(make_shape(B, L, D, lstm_lc<float>(), &s));
     return launch_newton<LstmCell, float, lstm_tile_arg<float>()>(s, u, dt, a, s0, st, tol, max_iters, ws, stream);
+}
+
+// ------------------------------------------------ segments of a sequence
+
+// One Newton pass over a segment (see segment.cuh): from s_in (NULL: the zero
+// guess), linearising the segment's first step at s_lin, with s_carry as the
+// state entering it; the segment's last-step states are copied to s_end.
+// Components are stacked: s_in, s_out [NS][B][Ls][D]; s_lin, s_carry, s_end [NS][B][D].
+pararnn_status segment_pass_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* s_in,
+                                  const float* s_lin, const float* s_carry, float* s_out, float* s_end, long long B,
+                                  long long L, long long D, void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(dt));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(s_in, "s_in", false));
+    TRY(check_ptr(s_lin, "s_lin", false));
+    TRY(check_ptr(s_carry, "s_carry", false));
+    TRY(check_ptr(s_out, "s_out", true));
+    TRY(check_ptr(s_end, "s_end", false));
+    Shape s;
+    TRY(make_shape(B, L, D, cell == 0 ? kLcGru : kLcLstm, &s));
+    TRY(check_workspace(ws, ws_bytes, solve_ws_bytes(cell, B, L, D)));
+    const int NS = cell == 0 ? 1 : 2;
+    const long long per = B * L * D, per0 = B * D;
+    if (s_in) {  // other CTAs overwrite what one still reads: no overlap
+        const uintptr_t i0 = reinterpret_cast<uintptr_t>(s_in), o0 = reinterpret_cast<uintptr_t>(s_out);
+        const uintptr_t len = uintptr_t(NS * per) * 4;
+        if (i0 < o0 + len && o0 < i0 + len) return fail(PARARNN_ERR_INVALID_ARG, "s_out overlaps s_in");
+    }
+    const float* s0[2] = {s_carry, s_carry && NS == 2 ? s_carry + per0 : nullptr};
+    float* st[2] = {s_out, NS == 2 ? s_out + per : nullptr};
+    const float* in[2] = {s_in ? s_in : s_out, s_in ? s_in + (NS - 1) * per : s_out + (NS - 1) * per};
+    const float* lin[2] = {s_lin, s_lin && NS == 2 ? s_lin + per0 : nullptr};
+    // no device-side decision: exactly one pass (tol < 0 is never met)
+    const float tol = -1.0f;
+    const int warm = s_in ? 1 : 0;
+    pararnn_status r;
+    if (cell == 0) {
+        if (dt == PARARNN_BF16) {
+            TRY(make_shape(B, L, D, gru_lc<uint16_t>(), &s));
+            r = launch_newton<GruCell, uint16_t, gru_tile_arg<uint16_t>()>(s, u, dt, a, s0, st, tol, 1, ws, stream, in,
+                                                                          lin, warm);
+        } else {
+            TRY(make_shape(B, L, D, gru_lc<float>(), &s));
+            r = launch_newton<GruCell, float, gru_tile_arg<float>()>(s, u, dt, a, s0, st, tol, 1, ws, stream, in, lin,
+                                                                    warm);
+        }
+    } else {
+        if (dt == PARARNN_BF16) {
+            TRY(make_shape(B, L, D, lstm_lc<uint16_t>(), &s));
+            r = launch_newton<LstmCell, uint16_t, lstm_tile_arg<uint16_t>()>(s, u, dt, a, s0, st, tol, 1, ws, stream,
+                                                                            in, lin, warm);
+        } else {
+            TRY(make_shape(B, L, D, lstm_lc<float>(), &s));
+            r = launch_newton<LstmCell, float, lstm_tile_arg<float>()>(s, u, dt, a, s0, st, tol, 1, ws, stream, in,
+                                                                      lin, warm);
+        }
+    }
+    TRY(r);
+    if (s_end) {
+        for (int q = 0; q < NS; ++q)
+            CUDA_TRY(cudaMemcpy2DAsync(s_end + q * per0, size_t(D) * 4, st[q] + (L - 1) * D, size_t(L) * D * 4,
+                                       size_t(D) * 4, size_t(B), cudaMemcpyDeviceToDevice, stream));
+    }
+    return PARARNN_OK;
+}
+
+pararnn_status segment_update_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* beta,
+                                    const float* unit, const float* carry, float* s_out, float* residual, long long B,
+                                    long long L, long long D, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_dtype(dt));
+    TRY(check_ptr(u, "u", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(beta, "beta", true));
+    TRY(check_ptr(unit, "unit", true));
+    TRY(check_ptr(carry, "carry", true));
+    TRY(check_ptr(s_out, "s_out", true));
+    if (!residual) return fail(PARARNN_ERR_INVALID_ARG, "residual is NULL");
+    Shape s;
+    TRY(make_shape(B, L, D, 1, &s));
+    const long long n = B * L * D;
+    const dim3 grid(unsigned((n + 255) / 256)), block(256);
+    unsigned* res = reinterpret_cast<unsigned*>(residual);
+    if (cell == 0) {
+        if (dt == PARARNN_BF16)
+            segment_update_kernel<GruCell, uint16_t><<<grid, block, 0, stream>>>(
+                static_cast<const uint16_t*>(u), a, beta, unit, carry, s_out, res, B, L, D);
+        else
+            segment_update_kernel<GruCell, float><<<grid, block, 0, stream>>>(static_cast<const float*>(u), a, beta,
+                                                                              unit, carry, s_out, res, B, L, D);
+    } else {
+        if (dt == PARARNN_BF16)
+            segment_update_kernel<LstmCell, uint16_t><<<grid, block, 0, stream>>>(
+                static_cast<const uint16_t*>(u), a, beta, unit, carry, s_out, res, B, L, D);
+        else
+            segment_update_kernel<LstmCell, float><<<grid, block, 0, stream>>>(static_cast<const float*>(u), a, beta,
+                                                                               unit, carry, s_out, res, B, L, D);
+    }
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
 }
 
 pararnn_status read_header(const void* ws, cudaStream_t stream, WsHeader* h)
@@ -904,6 +1024,64 @@ pararnn_status pararnn_lstm_step(const void* u, pararnn_dtype u_dtype, const flo
     if (overlap(c_next, h_next, n)) return fail(PARARNN_ERR_INVALID_ARG, "c_next and h_next overlap");
     return launch_step<LstmCell>(u, u_dtype, a, c_prev, h_prev, c_next, h_next, B, D,
                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------- segments of a sequence
+
+pararnn_status pararnn_gru_segment_pass(const void* u, pararnn_dtype u_dtype, const float* a, const float* h_in,
+                                        const float* h_lin, const float* h_carry, float* h_out, float* h_end,
+                                        int64_t B, int64_t L, int64_t D, void* workspace, size_t workspace_bytes,
+                                        pararnn_stream_t stream)
+{
+    return segment_pass_async(0, u, u_dtype, a, h_in, h_lin, h_carry, h_out, h_end, B, L, D, workspace,
+                              workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_lstm_segment_pass(const void* u, pararnn_dtype u_dtype, const float* a, const float* s_in,
+                                         const float* s_lin, const float* s_carry, float* s_out, float* s_end,
+                                         int64_t B, int64_t L, int64_t D, void* workspace, size_t workspace_bytes,
+                                         pararnn_stream_t stream)
+{
+    return segment_pass_async(1, u, u_dtype, a, s_in, s_lin, s_carry, s_out, s_end, B, L, D, workspace,
+                              workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_gru_segment_update(const void* u, pararnn_dtype u_dtype, const float* a, const float* beta,
+                                          const float* unit, const float* carry, float* h_out, float* residual,
+                                          int64_t B, int64_t L, int64_t D, pararnn_stream_t stream)
+{
+    return segment_update_async(0, u, u_dtype, a, beta, unit, carry, h_out, residual, B, L, D,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_lstm_segment_update(const void* u, pararnn_dtype u_dtype, const float* a, const float* beta,
+                                           const float* unit, const float* carry, float* s_out, float* residual,
+                                           int64_t B, int64_t L, int64_t D, pararnn_stream_t stream)
+{
+    return segment_update_async(1, u, u_dtype, a, beta, unit, carry, s_out, residual, B, L, D,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_segment_carries(const float* ends, const float* s0, float* carries, int n_segments,
+                                       int n_state, int64_t B, int64_t D, pararnn_stream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_ptr(ends, "ends", true));
+    TRY(check_ptr(s0, "s0", false));
+    TRY(check_ptr(carries, "carries", true));
+    if (n_segments < 1) return fail(PARARNN_ERR_INVALID_ARG, "n_segments must be >= 1 (got %d)", n_segments);
+    if (n_state != 1 && n_state != 2) return fail(PARARNN_ERR_INVALID_ARG, "n_state must be 1 or 2 (got %d)", n_state);
+    if (B < 1 || D < 1) return fail(PARARNN_ERR_INVALID_ARG, "B, D must be >= 1");
+    const long long BD = (long long)B * D;
+    const dim3 grid(unsigned((BD + 255) / 256)), block(256);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (n_state == 1)
+        segment_carries_kernel<1><<<grid, block, 0, st>>>(ends, s0, carries, n_segments, BD);
+    else
+        segment_carries_kernel<2><<<grid, block, 0, st>>>(ends, s0, carries, n_segments, BD);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
 }
 
 size_t pararnn_linear_scan_workspace_size(int64_t B, int64_t L, int64_t D) { return linear_scan_ws_bytes(B, L, D); }

@@ -104,6 +104,28 @@ def test_argument_checks_before_any_gpu_work(capi):
     assert lib.pararnn_read_pass_times(256, None, None, 4, ctypes.byref(n)) == E.ERR_INVALID_ARG
 
 
+def test_segment_checks(capi):
+    """The sequence-split pieces check their arguments before any launch."""
+    E, lib = capi, capi.lib
+    seg = lambda u=16, a=16, si=None, so=4096, B=1, L=8, D=16, ws=256, wsb=1 << 20: lib.pararnn_gru_segment_pass(
+        u, 1, a, si, None, None, so, None, B, L, D, ws, wsb, None)
+    assert seg(u=None) == E.ERR_INVALID_ARG
+    assert seg(so=None) == E.ERR_INVALID_ARG
+    assert seg(D=12) == E.ERR_UNSUPPORTED
+    assert seg(ws=None) == E.ERR_WORKSPACE
+    assert seg(si=4096, so=4096 + 64) == E.ERR_INVALID_ARG  # output overlaps the iterate it reads
+    assert "overlaps" in capi.last_error()
+    assert lib.pararnn_lstm_segment_pass(16, 1, 16, None, None, None, None, None, 1, 8, 16, 256, 1 << 20,
+                                         None) == E.ERR_INVALID_ARG
+    upd = lambda res=4096, D=16: lib.pararnn_gru_segment_update(16, 1, 16, 16, 16, 16, 16, res, 1, 8, D, None)
+    assert upd(res=None) == E.ERR_INVALID_ARG
+    assert upd(D=12) == E.ERR_UNSUPPORTED
+    car = lambda R=2, NS=1, B=1, D=16: lib.pararnn_segment_carries(16, None, 16, R, NS, B, D, None)
+    assert car(R=0) == E.ERR_INVALID_ARG
+    assert car(NS=3) == E.ERR_INVALID_ARG
+    assert car(B=0) == E.ERR_INVALID_ARG
+
+
 def test_decode_step_checks(capi):
     """The decode step refuses bad shapes, pointers and partial overlaps
     before any launch; an output that is its own previous state passes."""

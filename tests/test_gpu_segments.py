@@ -1,0 +1,79 @@
+"""GPU parity of the solve with the sequence split into segments (the
+multi-GPU sequence sharding), run here as R segments one after another on one
+GPU: the iterates are those of the single-GPU solve, so the states match it
+(1e-5) and the oracle's sequential states (1e-4), and the iteration count is
+the oracle's Newton count (+-1 where its residual is within 10x of tol)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nonlinear_rnn_newton_b200 import sharded as SH
+from nonlinear_rnn_newton_b200 import workloads as W
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+def P():
+    import nonlinear_rnn_newton_b200 as pkg
+    return pkg
+
+
+SPLITS = [[1000], [500, 500], [1, 333, 666], [128, 256, 7, 409, 200]]
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("lens", SPLITS, ids=lambda v: f"R{len(v)}")
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_segments_match_single_gpu_and_oracle(cuda, cell, lens, dt):
+    B, L, D = 3, sum(lens), 136
+    w = W.custom(cell, B, L, D, dt, h0_std=0.1)
+    x = W.make_inputs(w, seed=len(lens))
+    xd = x.to(cuda)
+    NS = 1 if cell == "gru" else 2
+    s0 = torch.zeros((NS, B, D), device=cuda)
+    if xd.h0 is not None:
+        s0[NS - 1] = xd.h0
+    edges = np.cumsum([0] + lens)
+    segs = [SH.Segment(cell, xd.u[:, edges[r]:edges[r + 1]].contiguous(), xd.a, r) for r in range(len(lens))]
+    it, res, st = SH.solve_segments(segs, SH.LocalComm(), s0, w.tol, w.max_iters)
+    Hs = torch.cat([sg.H for sg in segs], dim=2)
+    if cell == "gru":
+        h, it1, r1, st1 = P().pararnn_gru_solve(xd.u, xd.a, xd.h0)
+        one = h[None]
+        seq = oracle.gru_seq(x.u, x.a, x.h0)[None]
+        _, oit, _, _, hist = oracle.gru_newton(x.u, x.a, x.h0)
+    else:
+        c, h, it1, r1, st1 = P().pararnn_lstm_solve(xd.u, xd.a, None, xd.h0)
+        one = torch.stack([c, h])
+        sc, sh = oracle.lstm_seq(x.u, x.a, None, x.h0)
+        seq = np.stack([sc, sh])
+        *_, oit, _, _, hist = oracle.lstm_newton(x.u, x.a, None, x.h0)
+    torch.cuda.synchronize()
+    assert st == 0 and H.iters_agree(it, oit, hist, w.tol), (it, oit, hist)
+    assert float((Hs - one).abs().max()) <= 1e-5
+    assert H.max_abs(Hs.cpu(), seq) <= 1e-4
+
+
+def test_segment_stopping_rules(cuda):
+    """max_iters = 0 and a huge tol stop at the zero guess; max_iters = 1
+    gives the oracle's first iterate; each piece checks its arguments."""
+    w = W.custom("gru", 2, 300, 64, "f32", h0_std=0.1)
+    x = W.make_inputs(w, seed=3)
+    xd = x.to(cuda)
+    s0 = xd.h0[None].contiguous()
+    segs = [SH.Segment("gru", xd.u[:, :100].contiguous(), xd.a, 0),
+            SH.Segment("gru", xd.u[:, 100:].contiguous(), xd.a, 1)]
+    it, r, st = SH.solve_segments(segs, SH.LocalComm(), s0, max_iters=0)
+    h0, oit, ores, ost, hist = oracle.gru_newton(x.u, x.a, x.h0, max_iters=0)
+    assert it == 0 and st == 1 and abs(r - ores) <= 1e-6 * max(1.0, ores)
+    it, r, st = SH.solve_segments(segs, SH.LocalComm(), s0, tol=1e30)
+    assert it == 0 and st == 0
+    it, r, st = SH.solve_segments(segs, SH.LocalComm(), s0, tol=0.0, max_iters=1)
+    h1, *_ = oracle.gru_newton(x.u, x.a, x.h0, tol=0.0, max_iters=1)
+    Hs = torch.cat([sg.H for sg in segs], dim=2)[0]
+    assert it == 1 and st == 1 and H.max_abs(Hs.cpu(), h1) <= 1e-4
+    from nonlinear_rnn_newton_b200 import capi
+    with pytest.raises(capi.PararnnError):  # output overlapping the iterate it reads
+        P().pararnn_gru_segment_pass(segs[0].u, xd.a, segs[0].H, None, None, segs[0].H, None, segs[0].ws)

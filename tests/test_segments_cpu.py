@@ -1,0 +1,138 @@
+"""The host logic of the sequence-split solve (nonlinear_rnn_newton_b200.sharded)
+on CPU ranks (gloo, world size 2 and 3): every rank holds one segment, the
+segments' ends are all-gathered in segment order, the residual maximum is
+all-reduced, and the stopping decision is common.  The per-segment
+computations are a float64 stand-in written here from the method (one Newton
+pass over a segment from a linearisation point and a carry; the affine
+fix-up; the composition of the segments' maps), so the test checks the
+orchestration and the algebra, not the kernels (which the GPU tests check).
+Expected: the oracle's sequential states and its Newton iteration count."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+class Float64Segment:
+    """The interface of sharded.Segment, computed in float64 on the CPU."""
+
+    def __init__(self, cell, u, a, index):
+        self.cell, self.index, self.stream = cell, index, None
+        self.step, self.jac = cell.step, cell.jac
+        self.NS = cell.NS
+        self.u = u                                   # [B, Ls, G, D] float64
+        self.a = a.numpy()
+        self.ug = np.transpose(u.numpy(), (1, 2, 0, 3))  # [Ls, G, B, D]
+        B, Ls, G, D = u.shape
+        self.H = torch.zeros((self.NS, B, Ls, D), dtype=torch.float64)
+        self.P = np.zeros((1 + self.NS, self.NS, B, Ls, D))
+        self.ends = torch.zeros((1 + self.NS, self.NS, B, D), dtype=torch.float64)
+        self.lin = np.zeros((self.NS, B, D))
+        self.res = torch.zeros(1, dtype=torch.float64)
+
+    def _residual(self, Hn, prev0):
+        prev, r = prev0, 0.0
+        for l in range(Hn.shape[2]):
+            r = max(r, float(np.max(np.abs(Hn[:, :, l] - self.step(prev, self.ug[l], self.a)))))
+            prev = Hn[:, :, l]
+        return r
+
+    def start(self, s0):
+        self.H.zero_()
+        self.lin = s0.numpy().copy() if (self.index == 0 and s0 is not None) else np.zeros_like(self.lin)
+        self.res[0] = self._residual(self.H.numpy(), self.lin)
+
+    def passes(self, k):
+        Hk = self.H.numpy()
+        for j in range(1 + self.NS):
+            c = np.zeros_like(self.lin)
+            if j > 0:
+                c[j - 1] = 1.0
+            prev_k, s = self.lin, c
+            for l in range(Hk.shape[2]):
+                J = self.jac(prev_k, self.ug[l], self.a)
+                f = self.step(prev_k, self.ug[l], self.a)
+                o = f - np.einsum("qrbd,rbd->qbd", J, prev_k)
+                s = np.einsum("qrbd,rbd->qbd", J, s) + o
+                self.P[j, :, :, l] = s
+                prev_k = Hk[:, :, l]
+            self.ends[j] = torch.from_numpy(self.P[j, :, :, -1].copy())
+
+    def carries(self, ends, s0):
+        e = ends.numpy()
+        c = s0.numpy().copy() if s0 is not None else np.zeros(e.shape[2:])
+        out = np.empty((e.shape[0],) + c.shape)
+        for r in range(e.shape[0]):
+            out[r] = c
+            c = e[r, 0] + sum((e[r, 1 + j] - e[r, 0]) * c[j] for j in range(self.NS))
+        return torch.from_numpy(out)
+
+    def update(self, carry):
+        c = carry.numpy()
+        Hn = self.P[0] + sum((self.P[1 + j] - self.P[0]) * c[j][:, None, :] for j in range(self.NS))
+        self.res[0] = self._residual(Hn, c)
+        self.H = torch.from_numpy(Hn.copy())
+        self.lin = c.copy()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _draw(name, B, L, D):
+    from tests.user_cells import CELLS
+    cell = CELLS[name]
+    g = torch.Generator().manual_seed(5)
+    u = torch.randn((B, L, cell.G, D), generator=g, dtype=torch.float64)
+    a = torch.rand((cell.G, D), generator=g, dtype=torch.float64) - 0.5
+    s0 = torch.randn((cell.NS, B, D), generator=g, dtype=torch.float64) * 0.1
+    return cell, u, a, s0
+
+
+def _rank_main(rank, world, port, name, edges, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    from nonlinear_rnn_newton_b200 import sharded as SH
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cell, u, a, s0 = _draw(name, 2, edges[-1], 3)
+        seg = Float64Segment(cell, u[:, edges[rank]:edges[rank + 1]].contiguous(), a, rank)
+        it, r, st = SH.solve_segments([seg], SH.DistComm(), s0, tol=1e-10, max_iters=30, n_segments=world)
+        parts = [None] * world  # segments differ in length: gathered as objects, for the test only
+        dist.all_gather_object(parts, seg.H.numpy())
+        out[rank] = (it, r, st, np.concatenate(parts, axis=2))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name,edges", [("gru", [0, 23, 40]), ("lstm", [0, 9, 20, 31]), ("mixed", [0, 1, 16])])
+def test_ranks_solve_their_segments(name, edges):
+    from oracle import generic as OG
+    world = len(edges) - 1
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, name, edges, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    cell, u, a, s0 = _draw(name, 2, edges[-1], 3)
+    seq = OG.generic_seq(cell.step, u, a, s0, cell.NS)
+    _, oit, ores, ost, hist = OG.generic_newton(cell.step, cell.jac, u, a, s0, cell.NS, tol=1e-10, max_iters=30)
+    for r in range(world):
+        it, res, st, Hs = out[r]
+        assert (it, st) == (oit, ost)                  # same decision on every rank
+        assert abs(res - ores) <= 1e-12 + 1e-9 * ores
+        assert np.max(np.abs(Hs - seq)) < 1e-9
