@@ -63,12 +63,6 @@ struct NewtonParams {
     unsigned long long* desc;  // [n_tiles][desc_words] tagged words
     float* bnd;             // [2][NS][B][n_chunks][S*kDc]
     unsigned long long wait_ns;
-    // Segment passes (the sequence split across GPUs): the state the first
-    // step of chunk 0 is linearised at, per component (NULL = s0), and
-    // whether the first pass starts from the states the state tensor maps
-    // point at (1) instead of the zero guess (0).
-    const float* slin[2];
-    int warm;
 };
 
 

@@ -104,7 +104,10 @@ struct NewtonWsLayout {
     static constexpr bool fits = smem_bytes <= 232448;  // opt-in shared memory per CTA
 };
 
-template <class Cell, class UT, int CW>
+// Seg: the segment-pass form (warm start and a separate linearisation point
+// for chunk 0, read from the workspace header); a template parameter so that
+// the plain solve keeps its own code.
+template <class Cell, class UT, int CW, bool Seg = false>
 __global__ void __launch_bounds__(32 * (CW + 1), 1)
     newton_solve_ws_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_s0,
                            const __grid_constant__ CUtensorMap tm_s1, const __grid_constant__ CUtensorMap tm_a,
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 
     for (int k = 0;; ++k) {
         const int slot = k % 3;
-        const bool first = (k == 0) && !p.warm;  // the pass starts from H^0 = 0
+        const bool first = (k == 0) && !(Seg && hdr->seg_warm);  // the pass starts from H^0 = 0
         if (tid == 0) {
             if (blockIdx.x == 0) {
                 // slot (k+1)%3 was last used two passes ago; every CTA is past it
@@ -425,7 +428,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                         F4 x{{0.f, 0.f, 0.f, 0.f}};
                         if (w == 0) {
                             if (c == 0) {
-                                const float* lin = p.slin[q] ? p.slin[q] : p.s0[q];
+                                const float* lin = p.s0[q];
+                                if (Seg && hdr->seg_lin[q]) lin = reinterpret_cast<const float*>(hdr->seg_lin[q]);
                                 if (chv && lin) x = load4(lin + b * D + dch);
                             } else if (!first) {
                                 x = load4(sbnd + q * kDc + lane * kV);

@@ -286,7 +286,7 @@ pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid, int th
 
 // in: where the first pass reads the states (segment passes: the given
 // iterate; NULL = st); slin, warm: see NewtonParams.
-template <class Cell, class UT, int T>
+template <class Cell, class UT, int T, bool Seg = false>
 pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
                              float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream,
                              const float* const* in = nullptr, const float* const* slin = nullptr, int warm = 0)
@@ -295,7 +295,7 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
     constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
 #if PARARNN_WS
     using KL = NewtonWsLayout<Cell, UT, T>;  // T = compute warps (two steps each)
-    auto kern = newton_solve_ws_kernel<Cell, UT, T>;
+    auto kern = newton_solve_ws_kernel<Cell, UT, T, Seg>;
     constexpr int threads = KL::threads;
 #else
     using KL = NewtonLayout<Cell, UT, T>;    // T = steps per warp
@@ -314,7 +314,7 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
     TRY(map_state(&t0, src[0], s, KL::Lc));
     TRY(map_state(&t1, src[1], s, KL::Lc));
 
-    NewtonParams p{};
+    NewtonParams p;
     p.a = a;
     p.s0[0] = s0[0];
     p.s0[1] = s0[1];
@@ -332,9 +332,16 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
     p.desc = reinterpret_cast<unsigned long long*>(wsb + ly.desc);
     p.bnd = reinterpret_cast<float*>(wsb + ly.extra);
     p.wait_ns = kWaitLimitNs;
-    p.slin[0] = slin ? slin[0] : nullptr;
-    p.slin[1] = slin ? slin[1] : nullptr;
-    p.warm = warm;
+    if (Seg) {  // into the zeroed header (pageable source: consumed before the call returns)
+        struct {
+            unsigned long long lin[2];
+            int warm;
+        } seg = {{slin ? reinterpret_cast<unsigned long long>(slin[0]) : 0ull,
+                  slin ? reinterpret_cast<unsigned long long>(slin[1]) : 0ull},
+                 warm};
+        static_assert(offsetof(WsHeader, seg_warm) == offsetof(WsHeader, seg_lin) + 16, "header layout");
+        CUDA_TRY(cudaMemcpyAsync(wsb + offsetof(WsHeader, seg_lin), &seg, 20, cudaMemcpyHostToDevice, stream));
+    }
     if (warm && s.n_chunks > 1) {
         const long long n = (long long)NS * s.B * (s.n_chunks - 1) * (s.D / 4);
         bnd_gather_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(src[0], src[1], p.bnd, NS, s.B, s.L, s.D,
@@ -451,22 +458,22 @@ pararnn_status segment_pass_async(int cell, const void* u, pararnn_dtype dt, con
     if (cell == 0) {
         if (dt == PARARNN_BF16) {
             TRY(make_shape(B, L, D, gru_lc<uint16_t>(), &s));
-            r = launch_newton<GruCell, uint16_t, gru_tile_arg<uint16_t>()>(s, u, dt, a, s0, st, tol, 1, ws, stream, in,
-                                                                          lin, warm);
+            r = launch_newton<GruCell, uint16_t, gru_tile_arg<uint16_t>(), true>(s, u, dt, a, s0, st, tol, 1, ws,
+                                                                                stream, in, lin, warm);
         } else {
             TRY(make_shape(B, L, D, gru_lc<float>(), &s));
-            r = launch_newton<GruCell, float, gru_tile_arg<float>()>(s, u, dt, a, s0, st, tol, 1, ws, stream, in, lin,
-                                                                    warm);
+            r = launch_newton<GruCell, float, gru_tile_arg<float>(), true>(s, u, dt, a, s0, st, tol, 1, ws, stream, in,
+                                                                          lin, warm);
         }
     } else {
         if (dt == PARARNN_BF16) {
             TRY(make_shape(B, L, D, lstm_lc<uint16_t>(), &s));
-            r = launch_newton<LstmCell, uint16_t, lstm_tile_arg<uint16_t>()>(s, u, dt, a, s0, st, tol, 1, ws, stream,
-                                                                            in, lin, warm);
+            r = launch_newton<LstmCell, uint16_t, lstm_tile_arg<uint16_t>(), true>(s, u, dt, a, s0, st, tol, 1, ws,
+                                                                                  stream, in, lin, warm);
         } else {
             TRY(make_shape(B, L, D, lstm_lc<float>(), &s));
-            r = launch_newton<LstmCell, float, lstm_tile_arg<float>()>(s, u, dt, a, s0, st, tol, 1, ws, stream, in,
-                                                                      lin, warm);
+            r = launch_newton<LstmCell, float, lstm_tile_arg<float>(), true>(s, u, dt, a, s0, st, tol, 1, ws, stream,
+                                                                            in, lin, warm);
         }
     }
     TRY(r);

@@ -39,7 +39,14 @@ struct alignas(256) WsHeader {
     int passes;        // Newton passes run
     pararnn_result result;
     unsigned long long t_pass[kPassTimes];  // see kPassTimes (0 = not reached)
-    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result) - 8 * kPassTimes];
+    // Segment passes only (the sequence split across GPUs; written by the
+    // host after the header is zeroed): the state the first step of chunk 0
+    // is linearised at, per component (0 = s0), and whether the first pass
+    // starts from the states the state tensor maps point at (1) instead of
+    // the zero guess (0).
+    unsigned long long seg_lin[2];
+    int seg_warm;
+    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result) - 8 * kPassTimes - 8 * 2 - 4];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
 
