@@ -39,7 +39,8 @@ class Float64Segment:
     def _residual(self, Hn, prev0):
         prev, r = prev0, 0.0
         for l in range(Hn.shape[2]):
-            r = max(r, float(np.max(np.abs(Hn[:, :, l] - self.step(prev, self.ug[l], self.a)))))
+            # NaN kept, like the kernels' max.NaN (Python's max would drop it)
+            r = float(np.maximum(r, np.max(np.abs(Hn[:, :, l] - self.step(prev, self.ug[l], self.a)))))
             prev = Hn[:, :, l]
         return r
 
@@ -136,3 +137,28 @@ def test_ranks_solve_their_segments(name, edges):
         assert (it, st) == (oit, ost)                  # same decision on every rank
         assert abs(res - ores) <= 1e-12 + 1e-9 * ores
         assert np.max(np.abs(Hs - seq)) < 1e-9
+
+
+def test_stopping_paths_in_one_process():
+    """LocalComm (all segments in this process): max_iters = 0 and a huge tol
+    stop at the zero guess with its residual; max_iters = 1 gives the oracle's
+    first iterate; a NaN input stops with the non-finite status."""
+    from nonlinear_rnn_newton_b200 import sharded as SH
+    from oracle import generic as OG
+    cell, u, a, s0 = _draw("lstm", 2, 30, 3)
+    edges = [0, 7, 30]
+    segs = lambda uu: [Float64Segment(cell, uu[:, edges[r]:edges[r + 1]].contiguous(), a, r) for r in range(2)]
+    seq = segs(u)
+    it, r, st = SH.solve_segments(seq, SH.LocalComm(), s0, max_iters=0)
+    _, oit, ores, ost, hist = OG.generic_newton(cell.step, cell.jac, u, a, s0, cell.NS, max_iters=0)
+    assert (it, st) == (0, SH.NOT_CONVERGED) and abs(r - ores) <= 1e-12
+    it, r, st = SH.solve_segments(seq, SH.LocalComm(), s0, tol=1e30)
+    assert (it, st) == (0, SH.OK)
+    it, r, st = SH.solve_segments(seq, SH.LocalComm(), s0, tol=0.0, max_iters=1)
+    H1, *_ = OG.generic_newton(cell.step, cell.jac, u, a, s0, cell.NS, tol=0.0, max_iters=1)
+    Hs = np.concatenate([sg.H.numpy() for sg in seq], axis=2)
+    assert (it, st) == (1, SH.NOT_CONVERGED) and np.max(np.abs(Hs - H1)) < 1e-12
+    bad = u.clone()
+    bad[1, 20, 0, 2] = float("nan")
+    it, r, st = SH.solve_segments(segs(bad), SH.LocalComm(), s0)
+    assert st == SH.NONFINITE and r != r
