@@ -69,3 +69,23 @@ def test_cells_compile(capi, name, flags):
         capi.lib.pararnn_cell_destroy(h)
     else:
         assert st == capi.ERR_CUDA, capi.last_error()
+
+
+def _synthetic_step(G, NS):
+    body = "\n".join(f"    acc = acc + tanh(u[{g}] + a[{g}] * s[{g % NS}]);" for g in range(G))
+    outs = "\n".join(f"    out[{q}] = 0.5f * s[{q}] + 0.25f * sigmoid(acc + s[{(q + 1) % NS}]);" for q in range(NS))
+    return ("template <class T, class U>\n__device__ void recurrence_step(const T* s, const U* u, const U* a, T* out)\n"
+            "{\n    T acc = 0.0f;\n" + body + "\n" + outs + "\n}\n")
+
+
+@pytest.mark.parametrize("G,NS", [(2, 1), (4, 1), (1, 2), (3, 2)])
+def test_every_accepted_shape_compiles(capi, G, NS):
+    """The shapes the test cells do not cover (those cover (3,1), (4,2), (1,1),
+    (2,2)): the solve and adjoint instantiations compile and their tiles fit."""
+    import torch
+    st, h = create(capi, _synthetic_step(G, NS), G, NS)
+    if torch.cuda.is_available():
+        assert st == capi.OK, capi.last_error()
+        capi.lib.pararnn_cell_destroy(h)
+    else:
+        assert st == capi.ERR_CUDA, capi.last_error()
