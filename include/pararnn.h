@@ -166,12 +166,17 @@ PARARNN_API pararnn_status pararnn_read_result(const void* workspace, pararnn_st
  *
  * Its scratch is one fixed array of pararnn_gru_solve_noalloc_max_scratch()
  * bytes (16 MiB) per device, part of the library's module image; the call
- * allocates nothing (no cudaMalloc, no cudaFree, no other allocator).
+ * allocates nothing (no cudaMalloc, no cudaFree, no other allocator).  The
+ * array is held on every device where the library's module is loaded, until
+ * the process exits, whether or not this entry point is ever called.
  * Shapes whose pararnn_gru_workspace_size exceeds that return
- * PARARNN_ERR_WORKSPACE, before any device call, with the sizes in
- * pararnn_last_error().  The first call on a device looks up the scratch's
- * device address (cudaGetSymbolAddress, with that device current) and caches
- * it: make that first call before capturing `stream` into a graph.  The
+ * PARARNN_ERR_WORKSPACE, and invalid arguments their usual status, before
+ * any device call, with the reason in pararnn_last_error().  The first call
+ * on a device looks up the scratch's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it per device ordinal for the life of
+ * the process: make that first call before capturing `stream` into a graph,
+ * and do not call this entry point on a device after the host program has
+ * reset it (cudaDeviceReset), since the cached address then is stale.  The
  * scratch is shared by every call on the device, so calls that overlap in
  * time (other threads, or other streams not yet finished) race and must be
  * serialised by the caller.  Arguments, outputs and return values are those

@@ -246,11 +246,31 @@ def pararnn_gru_solve(u, a, h0=None, tol=1e-6, max_iters=10, h=None, workspace=N
     return dh, it.value, res.value, st
 
 
+def _gru_device_args(u, a, h0, h):
+    """Shape, dtype, layout and device checks of a ParaGRU call on device
+    tensors (the library checks pointers and sizes again, but it cannot see
+    a tensor's shape or device); returns (B, L, D)."""
+    if u.dim() != 4:
+        raise ValueError(f"u must be [B,L,3,D], got shape {tuple(u.shape)}")
+    B, L, G, D = u.shape
+    if G != 3:
+        raise ValueError("GRU gates must be [B,L,3,D]")
+    _dtype_code(u)
+    if not u.is_contiguous():
+        raise ValueError("u must be contiguous")
+    _need(a, "a", (3, D), device=u.device)
+    _need(h0, "h0", (B, D), device=u.device)
+    if h is None:
+        raise ValueError("h (the output) is required")
+    _need(h, "h", (B, L, D), device=u.device)
+    return B, L, D
+
+
 def pararnn_gru_solve_noalloc(u, a, h0, h, tol=1e-6, max_iters=10, stream=None):
     """ParaGRU Newton solve on the library's fixed device scratch (no
     workspace; device tensors only, h is the output).  Returns
     (iters, residual, status)."""
-    B, L, G, D = u.shape
+    B, L, D = _gru_device_args(u, a, h0, h)
     it = ctypes.c_int(0)
     res = ctypes.c_float(0.0)
     with torch.cuda.device(u.device):  # the scratch used is the current device's
@@ -268,7 +288,7 @@ def pararnn_gru_solve_noalloc_max_scratch():
 def pararnn_gru_solve_async(u, a, h0, h, workspace, tol=1e-6, max_iters=10, stream=None):
     """Queue a ParaGRU solve (device tensors only); read the outcome with
     pararnn_read_result(workspace)."""
-    B, L, G, D = u.shape
+    B, L, D = _gru_device_args(u, a, h0, h)
     st = lib.pararnn_gru_solve_async(_ptr(u), _dtype_code(u), _ptr(a), _ptr(h0), _ptr(h), B, L, D,
                                      float(tol), int(max_iters), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(),

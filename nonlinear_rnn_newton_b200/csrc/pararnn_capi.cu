@@ -54,17 +54,6 @@ pararnn_status fail(pararnn_status s, const char* fmt, ...)
         if (s_ != PARARNN_OK) return s_;          \
     } while (0)
 
-#ifndef PARARNN_WS
-#define PARARNN_WS 1
-#endif
-// Timesteps per warp in a tile (a tile has 8 warps).  Compile-time tuning
-// knobs; the workspace layout follows them.
-#ifndef PARARNN_GRU_ROWS
-#define PARARNN_GRU_ROWS 4
-#endif
-#ifndef PARARNN_LSTM_ROWS
-#define PARARNN_LSTM_ROWS 2
-#endif
 #ifndef PARARNN_ADJ_ROWS
 #define PARARNN_ADJ_ROWS 4
 #endif
@@ -78,19 +67,12 @@ constexpr size_t kSelftestWorkspace = 16384;
 #ifndef PARARNN_WS_LSTM_WARPS
 #define PARARNN_WS_LSTM_WARPS 7
 #endif
-#if PARARNN_WS
 // compute warps per CTA (two steps each); fp32 gates need twice the staging
 // space, so their tiles are half as long
 template <class UT> constexpr int gru_tile_arg() { return sizeof(UT) == 2 ? PARARNN_WS_GRU_WARPS : PARARNN_WS_GRU_WARPS / 2; }
 template <class UT> constexpr int lstm_tile_arg() { return sizeof(UT) == 2 ? PARARNN_WS_LSTM_WARPS : PARARNN_WS_LSTM_WARPS / 2; }
 template <class UT> constexpr int gru_lc() { return 2 * gru_tile_arg<UT>(); }
 template <class UT> constexpr int lstm_lc() { return 2 * lstm_tile_arg<UT>(); }
-#else
-template <class UT> constexpr int gru_tile_arg() { return PARARNN_GRU_ROWS; }
-template <class UT> constexpr int lstm_tile_arg() { return PARARNN_LSTM_ROWS; }
-template <class UT> constexpr int gru_lc() { return kWarps * PARARNN_GRU_ROWS; }
-template <class UT> constexpr int lstm_lc() { return kWarps * PARARNN_LSTM_ROWS; }
-#endif
 // workspace sizing uses the shortest tile (most tiles) of either input dtype
 constexpr int kLcGru = gru_lc<float>() < gru_lc<uint16_t>() ? gru_lc<float>() : gru_lc<uint16_t>();
 constexpr int kLcLstm = lstm_lc<float>() < lstm_lc<uint16_t>() ? lstm_lc<float>() : lstm_lc<uint16_t>();
@@ -293,15 +275,9 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
 {
     constexpr int NS = Cell::NS;
     constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
-#if PARARNN_WS
     using KL = NewtonWsLayout<Cell, UT, T>;  // T = compute warps (two steps each)
     auto kern = newton_solve_ws_kernel<Cell, UT, T, Seg>;
     constexpr int threads = KL::threads;
-#else
-    using KL = NewtonLayout<Cell, UT, T>;    // T = steps per warp
-    auto kern = newton_solve_kernel<Cell, UT, T>;
-    constexpr int threads = kThreads;
-#endif
     // the TMA boxes must be exactly the kernel's tile
     if (s.Lc != KL::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, KL::Lc);
     const ScanLayout ly = scan_layout(s, desc_words, solve_bnd_bytes(s, NS));
@@ -352,14 +328,10 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
 
     int grid = 0;
     TRY(resident_grid(kern, KL::smem_bytes, s.n_tiles, &grid, threads));
-#if PARARNN_WS
     CUtensorMap ta, tb;
     TRY(map_weights(&ta, a, Cell::G, s));
     TRY(map_bnd(&tb, p.bnd, NS, s));
     void* args[] = {(void*)&tu, (void*)&t0, (void*)&t1, (void*)&ta, (void*)&tb, (void*)&p};
-#else
-    void* args[] = {(void*)&tu, (void*)&t0, (void*)&t1, (void*)&p};
-#endif
     CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(threads), args,
                                          KL::smem_bytes, stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -379,11 +351,12 @@ size_t solve_ws_bytes(int cell, long long B, long long L, long long D)
     return scan_layout(s, TileDesc<Aff<2>, 2>::words, solve_bnd_bytes(s, 2)).total;
 }
 
-pararnn_status solve_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* c0, const float* h0,
-                           float* c, float* h, long long B, long long L, long long D, float tol, int max_iters,
-                           void* ws, size_t ws_bytes, cudaStream_t stream)
+// Host-side argument checks of a solve (everything but the workspace); no
+// device call.
+pararnn_status solve_args(int cell, const void* u, pararnn_dtype dt, const float* a, const float* c0, const float* h0,
+                          const float* c, const float* h, long long B, long long L, long long D, float tol,
+                          int max_iters)
 {
-    t_err[0] = '\0';
     TRY(check_dtype(dt));
     TRY(check_ptr(u, "u", true));
     TRY(check_ptr(a, "a", true));
@@ -396,7 +369,16 @@ pararnn_status solve_async(int cell, const void* u, pararnn_dtype dt, const floa
     if (!(tol >= 0.0f) || !std::isfinite(tol)) return fail(PARARNN_ERR_INVALID_ARG, "tol must be finite and >= 0");
     if (max_iters < 0) return fail(PARARNN_ERR_INVALID_ARG, "max_iters must be >= 0");
     Shape s;
-    TRY(make_shape(B, L, D, cell == 0 ? kLcGru : kLcLstm, &s));
+    return make_shape(B, L, D, cell == 0 ? kLcGru : kLcLstm, &s);
+}
+
+pararnn_status solve_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* c0, const float* h0,
+                           float* c, float* h, long long B, long long L, long long D, float tol, int max_iters,
+                           void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(solve_args(cell, u, dt, a, c0, h0, c, h, B, L, D, tol, max_iters));
+    Shape s;
     TRY(check_workspace(ws, ws_bytes, solve_ws_bytes(cell, B, L, D)));
     if (cell == 0) {
         const float* s0[2] = {h0, nullptr};
@@ -852,6 +834,9 @@ pararnn_status pararnn_gru_solve_noalloc(const void* u, pararnn_dtype u_dtype, c
                                          pararnn_stream_t stream, int* iters_out, float* residual_out)
 {
     t_err[0] = '\0';
+    // every argument check happens here, on the host, before the scratch
+    // lookup (which is the first device call)
+    TRY(solve_args(0, u, u_dtype, a, nullptr, h0, nullptr, h, B, L, D, tol, max_iters));
     const size_t need = pararnn_gru_workspace_size(B, L, D);
     if (need > kNoAllocScratchBytes)
         return fail(PARARNN_ERR_WORKSPACE,
