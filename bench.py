@@ -1,18 +1,25 @@
 """Benchmark of the ParaRNN Newton solve on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-cpu-baseline] [--sweep] [--decode] [--cells]
-                    [--seq-segments R1,R2,...]
+                    [--workload NAME] [--no-extras] [--no-cpu-baseline]
+                    [--decode] [--cells] [--seq-segments R1,R2,...]
 
 A step is one pass of the whole hot path over the workload through the C ABI:
 one full Newton solve (every iteration until convergence, the convergence
 test included) -- followed, for the training workload, by the reverse-time
-adjoint -- with inputs resident in HBM.  Default workload: ParaGRU, bf16 gate
-pre-activations / fp32 state, B=8, L=4096, D=1024 (u ~ N(0,1),
-a ~ U(-0.5,0.5), h0 ~ N(0,0.1), seed = rank).  Metric: tokens*channels per
-second = B*L*D / step time.  Under torchrun every rank solves its own
-independent problem (no collective on the data path) and the time is the max
-over ranks.
+adjoint -- with inputs resident in HBM.  The headline workload is the largest
+single-GPU Newton solve: ParaGRU, bf16 gate pre-activations / fp32 state,
+B=1, L=65536, D=2048 (u ~ N(0,1), a ~ U(-0.5,0.5), h0 ~ N(0,0.1),
+seed = rank).  Metric: tokens*channels per second = B*L*D / step time.
+Under torchrun every rank solves its own independent problem (no collective
+on the data path) and the time is the max over ranks.
+
+On one GPU the same line also carries, under "configs", every other solve
+workload (ParaGRU and ParaLSTM at B=8, L=4096, D=1024; the B=1, D=2048
+sequence-length sweep with the sequential GPU kernel and the plain linear scan
+at each L; the ParaLSTM training step, solve plus adjoint, at B=4, L=16384,
+D=2048), each with its roofline and per-pass figures, and the CPU oracle's
+sequential stepping timed on all host cores and on one core.
 
 Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle on a
 bounded sample of the same workload instead (the reference arm; rank 0 only).
@@ -294,34 +301,56 @@ def time_baselines(w, xd, out, stream, dev, reps=5):
     return res
 
 
-def run_sweep(dev, stream, reps=10):
-    """The sequence-length sweep (B=1, D=2048): Newton solve, sequential GPU
-    kernel and linear scan at each L.  L <= 2048 fits in L2 (flagged)."""
-    import nonlinear_rnn_newton_b200 as P
+def measure(w, dev, stream, reps=10, warmup=3, baselines=True):
+    """One workload at full size: `reps` back-to-back steps after `warmup`,
+    CUDA events around every solve (and adjoint), the solve's per-pass device
+    timestamps, and (GRU) the two GPU baselines on the same input.  Inputs
+    exceed L2 (flagged where they do not)."""
     peak, _ = hbm_peak()
-    out = []
-    for w in W.GRU_SWEEP:
-        xd = W.make_inputs(w, seed=0).to(dev)
-        st = Step(w, xd, dev, stream)
-        for _ in range(3):
-            st()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            st()
-        e1.record(stream)
-        stream.synchronize()
-        ms = e0.elapsed_time(e1) / reps
-        r = st.result()
-        gbs = solve_bytes(w, r[1]) / (ms * 1e-3) / 1e9
-        base = time_baselines(w, xd, st.out[0], stream, dev)
-        out.append({"workload": w.name, "L": w.L, "ms": ms, "value": w.N / (ms * 1e-3), "iters": r[1],
-                    "status": r[0], "gbs": gbs, "frac": gbs / peak,
-                    "l2_resident": w.N * (w.G * 2 + 4) < 126e6,
-                    "sequential_gpu_ms": base["sequential_gpu"]["ms"],
-                    "linear_scan_gpu_ms": base["linear_scan_gpu"]["ms"]})
-        del st, xd
-        torch.cuda.empty_cache()
+    xd = W.make_inputs(w, seed=0).to(dev)
+    st = Step(w, xd, dev, stream)
+    for _ in range(warmup):
+        st()
+    nev = 3 if w.train else 2
+    evs = events(reps, nev)
+    for i in range(reps):
+        st(evs[i])
+    stream.synchronize()
+    r = st.result()
+    if r[0] not in (0, 1):
+        raise SystemExit(f"{w.name}: solve failed: status {r[0]}")
+    solve_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    step_ms = statistics.mean(e[0].elapsed_time(e[-1]) for e in evs)
+    algo = solve_bytes(w, r[1])
+    out = {"workload": w.name, "cell": w.cell, "B": w.B, "L": w.L, "D": w.D, "u_dtype": w.u_dtype,
+           "ms_per_step": step_ms, "value": w.N / (step_ms * 1e-3), "unit": UNIT, "iters": r[1],
+           "status": r[0], "residual": r[2],
+           "l2_resident": solve_bytes(w, 1) < 126e6,
+           "roofline": {"bound": "hbm", "kernel": "newton_solve_ws_kernel", "kernel_ms_mean": solve_ms,
+                        "algorithmic_bytes_per_launch": algo, "achieved": algo / (solve_ms * 1e-3) / 1e9,
+                        "peak": peak, "unit": "GB/s", "frac": algo / (solve_ms * 1e-3) / 1e9 / peak,
+                        "traffic": profile_traffic("newton_solve_ws_kernel", w.name),
+                        "per_pass": per_pass(w, st.pass_times(), peak)}}
+    if w.train:
+        adj_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        ab = adjoint_bytes(w)
+        out["adjoint"] = {"kernel": "adjoint_kernel", "kernel_ms_mean": adj_ms, "algorithmic_bytes_per_launch": ab,
+                          "achieved": ab / (adj_ms * 1e-3) / 1e9, "frac": ab / (adj_ms * 1e-3) / 1e9 / peak,
+                          "traffic": profile_traffic("adjoint_kernel", w.name)}
+    if baselines and w.cell == "gru":
+        out["baselines"] = time_baselines(w, xd, st.out[0], stream, dev)
+    del st, xd
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_configs(headline, dev, stream):
+    """Every solve workload except the headline, one after another."""
+    out = {}
+    for w in (W.GRU, W.LSTM) + W.GRU_SWEEP + (W.LSTM_TRAIN,):
+        if w.name == headline.name:
+            continue
+        out[w.name] = measure(w, dev, stream)
     return out
 
 
@@ -451,64 +480,89 @@ def oracle_sample(w, x, rows, chans):
     return u, a, h0, dh, rows * w.L * chans
 
 
-def oracle_threads(w):
-    """Threads the oracle as it stands uses on this workload: its Newton solve
-    is one serial loop; its BPTT (training workload) runs OpenMP over channels."""
+def host_cores():
+    """Threads the oracle's OpenMP loops use on this host (its default: one
+    per core the process may run on)."""
     import oracle
-    return oracle.max_threads() if w.train else 1
+    return oracle.max_threads()
 
 
-def time_oracle(w, x, rows, chans, threads):
-    """Seconds of the oracle's Newton solve (plus BPTT for the training
-    workload) on the sample; the input widening to fp64 happens before the
-    clock starts."""
+def widen(u, a, h0):
+    return (u.double().numpy(), a.double().numpy(), None if h0 is None else h0.double().numpy())
+
+
+def time_oracle_seq(w, x, rows, chans, threads):
+    """Tokens*channels/s of the oracle's sequential stepping (the plain
+    definition of the solve's result: fp64 C, OpenMP over the independent
+    channels) on `threads` threads, on a sample of the workload; the fp64
+    widening of the inputs happens before the clock starts."""
     import numpy as np
 
     import oracle
     oracle.set_threads(threads)
-    u, a, h0, dh, n = oracle_sample(w, x, rows, chans)
-    u64, a64 = u.double().numpy(), a.double().numpy()
-    h064 = None if h0 is None else h0.double().numpy()
-    dh64 = None if dh is None else dh.double().numpy()
+    u, a, h0, _, n = oracle_sample(w, x, rows, chans)
+    u64, a64, h064 = widen(u, a, h0)
     t0 = time.perf_counter()
     if w.cell == "gru":
-        h, it, _, _, _ = oracle.gru_newton(u64, a64, h064, tol=w.tol, max_iters=w.max_iters)
-        if dh64 is not None:
-            oracle.gru_bptt(u64, a64, h064, dh64)
+        h = oracle.gru_seq(u64, a64, h064)
     else:
-        c, h, it, _, _, _ = oracle.lstm_newton(u64, a64, None, h064, tol=w.tol, max_iters=w.max_iters)
-        if dh64 is not None:
-            oracle.lstm_bptt(u64, a64, None, h064, dh64)
+        _, h = oracle.lstm_seq(u64, a64, None, h064)
     dt = time.perf_counter() - t0
     assert np.isfinite(h).all()
-    what = "Newton solve" + (" + BPTT" if dh64 is not None else "")
-    how = "serial Newton" + (f", BPTT on {threads} OpenMP threads" if dh64 is not None else "")
-    desc = (f"oracle {what} (fp64 C, {how}) on batch rows 0..{min(rows, w.B) - 1}"
-            f", channels 0..{min(chans, w.D) - 1} of the workload (B={min(rows, w.B)}, L={w.L}, "
-            f"D={min(chans, w.D)}; {it} iterations); fp64 widening of the inputs excluded")
+    desc = (f"oracle sequential stepping (fp64 C, OpenMP over channels, {threads} thread(s)) on batch rows "
+            f"0..{min(rows, w.B) - 1}, channels 0..{min(chans, w.D) - 1} of the workload (B={min(rows, w.B)}, "
+            f"L={w.L}, D={min(chans, w.D)}); fp64 widening of the inputs excluded")
     return n / dt, dt, desc
 
 
-def cpu_sample_shape(w):
-    """About 10-30 s of CPU work: the whole problem when it is cfg-1-sized,
-    else a slice of its channels."""
-    if w.N <= 40_000_000:
-        return w.B, w.D
-    return 1, max(128, min(w.D, 40_000_000 // (w.B * w.L)))
+def time_oracle_newton(w, x, rows, chans):
+    """Tokens*channels/s of the oracle's serial Newton solve (one thread: the
+    oracle's Newton is one serial loop) on a sample of the workload."""
+    import numpy as np
+
+    import oracle
+    oracle.set_threads(1)
+    u, a, h0, _, n = oracle_sample(w, x, rows, chans)
+    u64, a64, h064 = widen(u, a, h0)
+    t0 = time.perf_counter()
+    if w.cell == "gru":
+        h, it, _, _, _ = oracle.gru_newton(u64, a64, h064, tol=w.tol, max_iters=w.max_iters)
+    else:
+        _, h, it, _, _, _ = oracle.lstm_newton(u64, a64, None, h064, tol=w.tol, max_iters=w.max_iters)
+    dt = time.perf_counter() - t0
+    assert np.isfinite(h).all()
+    desc = (f"oracle serial Newton (fp64 C, 1 thread, {it} iterations) on batch row 0, channels "
+            f"0..{min(chans, w.D) - 1} (B=1, L={w.L}, D={min(chans, w.D)})")
+    return n / dt, dt, desc
+
+
+def cpu_baselines(w, x):
+    """The CPU oracle beside the GPU numbers: its sequential stepping on all
+    host cores (128 channels per thread, at most 1024 channels: a few seconds
+    of CPU work) and on one core (128 channels), and its serial Newton on one
+    core (64 channels)."""
+    cores = host_cores()
+    v, secs, desc = time_oracle_seq(w, x, 1, min(w.D, 1024, 128 * cores), cores)
+    v1, secs1, desc1 = time_oracle_seq(w, x, 1, 128, 1)
+    vn, secsn, descn = time_oracle_newton(w, x, 1, 64)
+    return {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc, "seconds": secs,
+            "one_core": {"value": v1, "unit": UNIT, "cores": 1, "sample": desc1, "seconds": secs1},
+            "serial_newton_one_core": {"value": vn, "unit": UNIT, "cores": 1, "sample": descn, "seconds": secsn}}
 
 
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    threads = oracle_threads(w)
+    cores = host_cores()
     x = W.make_inputs(w, seed=0)
-    # each step: one batch row (all channels) -- a bounded sample so that the
-    # whole run stays within minutes
-    chans = w.D if w.L * w.D <= 8_400_000 else max(128, 8_400_000 // w.L)
+    # each step: the oracle's sequential stepping on all host cores over one
+    # batch row and 32 channels per thread (at most all of them) -- a bounded
+    # sample, so that the whole run stays within minutes
+    chans = min(w.D, 32 * cores)
     vals, desc = [], ""
     for i in range(args.warmup + args.steps):
-        v, _, desc = time_oracle(w, x, 1, chans, threads)
+        v, _, desc = time_oracle_seq(w, x, 1, chans, cores)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
@@ -517,7 +571,7 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * (w.L * chans) / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -580,18 +634,22 @@ def run_e2e(w, x, dev, steps, nbuf=2):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
+HEADLINE = W.BY_NAME["gru_bf16_B1_L65536_D2048"]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=W.GRU.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--workload", default=HEADLINE.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--no-extras", action="store_true", help="only the headline workload (the other solve "
+                    "workloads run by default on one GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--baselines", type=int, default=1, help="also time the sequential GPU kernel and "
-                    "the plain linear scan on the same input (GRU workloads)")
-    ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep (B=1, D=2048)")
+                    "the plain linear scan on the headline's input (GRU workloads)")
     ap.add_argument("--decode", action="store_true", help="add the decode-step timings (CUDA graph of steps)")
     ap.add_argument("--cells", action="store_true", help="add the runtime-compiled user cells (GRU, LSTM sources)")
     ap.add_argument("--seq-segments", default="", help="comma list of R: the solve with each sequence split into "
@@ -659,7 +717,8 @@ def main():
     if w.train:
         ab = adjoint_bytes(w)
         adjoint = {"kernel_ms_mean": adj_ms, "algorithmic_bytes_per_launch": ab,
-                   "achieved": ab / (adj_ms * 1e-3) / 1e9, "frac": ab / (adj_ms * 1e-3) / 1e9 / peak}
+                   "achieved": ab / (adj_ms * 1e-3) / 1e9, "frac": ab / (adj_ms * 1e-3) / 1e9 / peak,
+                   "traffic": profile_traffic("adjoint_kernel", w.name)}
 
     e2e = None
     if args.e2e_steps > 0:
@@ -672,21 +731,21 @@ def main():
     baselines = None
     if args.baselines and w.cell == "gru":
         baselines = time_baselines(w, xd, step.out[0], stream, dev)
+    del step, xd
+    torch.cuda.empty_cache()
 
-    sweep = run_sweep(dev, stream) if (args.sweep and rank == 0) else None
-    decode = run_decode(dev, stream) if (args.decode and rank == 0) else None
-    cells = run_cells(dev, stream) if (args.cells and rank == 0) else None
+    # the other workloads and the CPU oracle: one GPU only (under torchrun
+    # the ranks would wait for rank 0 at the process group's end)
+    solo = rank == 0 and world == 1
+    configs = run_configs(w, dev, stream) if (solo and not args.no_extras) else None
+    decode = run_decode(dev, stream) if (args.decode and solo) else None
+    cells = run_cells(dev, stream) if (args.cells and solo) else None
     segments = None
-    if args.seq_segments and rank == 0:
-        segments = run_segments(w, xd, dev, stream, [int(v) for v in args.seq_segments.split(",")])
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        threads = oracle_threads(w)
-        rows, chans = cpu_sample_shape(w)
-        v, secs, desc = time_oracle(w, x, rows, chans, threads)
-        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
-               "seconds": secs}
+    if args.seq_segments and solo:
+        xs = x.to(dev)
+        segments = run_segments(w, xs, dev, stream, [int(v) for v in args.seq_segments.split(",")])
+        del xs
+    cpu = cpu_baselines(w, x) if (solo and not args.no_cpu_baseline) else None
 
     if rank == 0:
         line = {
@@ -706,7 +765,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "baselines": baselines,
-            "sweep": sweep,
+            "configs": configs,
             "decode": decode,
             "user_cells": cells,
             "seq_segments": segments,

@@ -20,7 +20,7 @@ def test_reference_arm_prints_the_contract_line():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
-    assert line["config"]["workload"] == "gru_bf16_B8_L4096_D1024"
+    assert line["config"]["workload"] == "gru_bf16_B1_L65536_D2048"
 
 
 def test_pass_bytes_sum_to_solve_bytes():
