@@ -267,6 +267,65 @@ __device__ __forceinline__ F4 load4(const float* p)
     return r;
 }
 
+// N = 4 or 2 consecutive values (16- or 8-byte accesses; bf16 widened).
+template <int N>
+struct FV {
+    float v[N];
+};
+
+template <int N>
+__device__ __forceinline__ FV<N> loadv(const float* p)
+{
+    FV<N> r;
+    if constexpr (N == 4) {
+        const float4 w = *reinterpret_cast<const float4*>(p);
+        r.v[0] = w.x;
+        r.v[1] = w.y;
+        r.v[2] = w.z;
+        r.v[3] = w.w;
+    } else {
+        static_assert(N == 2, "2 or 4 values");
+        const float2 w = *reinterpret_cast<const float2*>(p);
+        r.v[0] = w.x;
+        r.v[1] = w.y;
+    }
+    return r;
+}
+
+template <int N>
+__device__ __forceinline__ FV<N> loadv(const uint16_t* p)
+{
+    FV<N> r;
+    if constexpr (N == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p);
+        r.v[0] = __uint_as_float(w.x << 16);
+        r.v[1] = __uint_as_float(w.x & 0xffff0000u);
+        r.v[2] = __uint_as_float(w.y << 16);
+        r.v[3] = __uint_as_float(w.y & 0xffff0000u);
+    } else {
+        static_assert(N == 2, "2 or 4 values");
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+        r.v[0] = __uint_as_float(w << 16);
+        r.v[1] = __uint_as_float(w & 0xffff0000u);
+    }
+    return r;
+}
+
+template <int N>
+__device__ __forceinline__ void storev(float* p, const float* v)
+{
+    if constexpr (N == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+}
+
+// streaming store to global memory (kept in L2 only)
+template <int N>
+__device__ __forceinline__ void stcgv(float* p, const float* v)
+{
+    if constexpr (N == 4) __stcg(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
+    else __stcg(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
+}
+
 __device__ __forceinline__ F4 ldcg4(const float* p)
 {
     float4 w = __ldcg(reinterpret_cast<const float4*>(p));

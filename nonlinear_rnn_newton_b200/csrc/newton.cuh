@@ -34,6 +34,7 @@ struct NewtonParams {
     unsigned long long* desc;  // [n_tiles][desc_words] tagged words
     float* bnd;             // [2][NS][B][n_chunks][S*kDc]
     unsigned long long wait_ns;
+    int lb_walk;            // look-backs step over aggregates (many groups of a sequence in flight)
 };
 
 

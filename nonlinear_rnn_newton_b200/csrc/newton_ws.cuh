@@ -43,21 +43,23 @@ namespace pararnn {
 #endif
 constexpr int kStages = PARARNN_WS_STAGES;  // TMA ring
 constexpr int kWork = 2;    // per-tile work buffers (tiles n-1 and n are live)
-// A ticket hands out `group` consecutive chunks of one sequence; they run
-// back to back in one CTA, so only the first of them looks back across CTAs
-// (the others take their carry from the tile before, in registers).  This
-// halves the chain of cross-CTA look-backs along a sequence.  The group's
-// second tile is prepared while the first one's look-back read is in flight
-// and its inclusive value is published together with the first one's, so the
-// chain advances two chunks per look-back.  (Longer groups would need the
-// control warp to wait for folds the compute warps can only produce after
-// the first tile's carry, so two is the longest that pays.)
-#ifndef PARARNN_WS_GROUP_GRU
-#define PARARNN_WS_GROUP_GRU 2
-#endif
-#ifndef PARARNN_WS_GROUP_LSTM
-#define PARARNN_WS_GROUP_LSTM 2
-#endif
+// A ticket hands out a group of kGroup = 2 consecutive chunks of one
+// sequence; they run back to back in one CTA.  The decoupled look-back works
+// on groups: the group's aggregate (the composition of its two tiles' maps)
+// and its inclusive value (the state leaving it) are published in one
+// descriptor per group, numbered like the tickets (group chunk * B * S +
+// sequence), so a look-back steps back one group per read and never waits on
+// a tile that publishes nothing.  The second tile takes its carry from the
+// first in registers.  (Longer groups would need the control warp to wait
+// for folds the compute warps can only produce after the first tile's carry,
+// so two is the longest that can be prepared ahead.)
+constexpr int kGroup = 2;
+
+// Look-back descriptors a solve uses: one per group of every sequence.
+__host__ __device__ constexpr long long solve_desc_count(int n_chunks, long long BS)
+{
+    return (long long)((n_chunks + kGroup - 1) / kGroup) * BS;
+}
 
 __device__ __forceinline__ float max_keep_nan(float a, float b)
 {
@@ -66,6 +68,7 @@ __device__ __forceinline__ float max_keep_nan(float a, float b)
     return r;
 }
 
+// CW: compute warps = row pairs (two steps each) in a tile.
 template <class Cell, class UT, int CW>
 struct NewtonWsLayout {
     static constexpr int G = Cell::G;
@@ -96,10 +99,11 @@ struct NewtonWsLayout {
     // misc: barriers (full, empty per stage; aggr, carry per work buffer), a
     // job (ticket, chunk, batch row, first channel) per stage, 8 flags,
     // 2*(CW+1) residual slots
+    static constexpr int CWT = CW;  // compute warps
     static constexpr size_t misc_bytes =
-        a128((2 * kStages + 2 * kWork) * 8 + kStages * 16 + 8 * 4 + 2 * (CW + 1) * 4);
+        a128((2 * kStages + 2 * kWork) * 8 + kStages * 16 + 8 * 4 + 2 * (CWT + 1) * 4);
     static constexpr size_t smem_bytes = off_misc + misc_bytes;
-    static constexpr int threads = 32 * (CW + 1);
+    static constexpr int threads = 32 * (CWT + 1);
     static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
     static constexpr bool fits = smem_bytes <= 232448;  // opt-in shared memory per CTA
 };
@@ -107,7 +111,7 @@ struct NewtonWsLayout {
 // Seg: the segment-pass form (warm start and a separate linearisation point
 // for chunk 0, read from the workspace header); a template parameter so that
 // the plain solve keeps its own code.
-template <class Cell, class UT, int CW, bool Seg = false>
+template <class Cell, class UT, int CW, bool Seg = false, int LB = 2>
 __global__ void __launch_bounds__(32 * (CW + 1), 1)
     newton_solve_ws_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_s0,
                            const __grid_constant__ CUtensorMap tm_s1, const __grid_constant__ CUtensorMap tm_a,
@@ -119,8 +123,11 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
     using Rows2 = typename Packed::Rows2;
     using Map2 = typename Packed::Map2;
     using Jac2 = typename Packed::Jac2;
-    constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc;
-    constexpr int kGroup = NS == 1 ? PARARNN_WS_GROUP_GRU : PARARNN_WS_GROUP_LSTM;
+    constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc, CWT = LY::CWT;
+    constexpr int CV = kV, NP = kV / 2;  // channels and channel pairs of a compute lane
+    // look-backs step back over aggregates (LB = 1), wait for inclusive
+    // values (LB = 0), or follow p.lb_walk (LB = 2)
+    const bool walk = LB == 2 ? p.lb_walk != 0 : LB == 1;
     static_assert(LY::fits, "shared memory");
 
     extern __shared__ __align__(128) unsigned char smem[];
@@ -130,14 +137,14 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
     uint64_t* bar_carry = bar_aggr + kWork;                                  // [kWork]
     int4* s_job = reinterpret_cast<int4*>(bar_carry + kWork);                // [kStages]
     int* s_int = reinterpret_cast<int*>(s_job + kStages);                    // misc flags
-    float* s_red = reinterpret_cast<float*>(s_int + 8);                      // [2 * (CW + 1)]
+    float* s_red = reinterpret_cast<float*>(s_int + 8);                      // [2 * (CWT + 1)]
     auto stage_at = [&](int i) { return smem + i * LY::stage_bytes; };
     auto work_at = [&](int i) { return smem + LY::off_work + i * LY::work_bytes; };
 
     const int tid = threadIdx.x;
     const int w = tid >> 5;
     const int lane = tid & 31;
-    const bool ctl = (w == CW);
+    const bool ctl = (w == CWT);
     WsHeader* hdr = p.hdr;
     int* err = &hdr->error;
     const long long D = p.D, L = p.L;
@@ -170,14 +177,14 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     mbar_inval(&bar_empty[i]);
                 }
                 mbar_init(&bar_full[i], 1);
-                mbar_init(&bar_empty[i], CW);
+                mbar_init(&bar_empty[i], CWT);
             }
             for (int i = 0; i < kWork; ++i) {
                 if (k > 0) {
                     mbar_inval(&bar_aggr[i]);
                     mbar_inval(&bar_carry[i]);
                 }
-                mbar_init(&bar_aggr[i], CW);
+                mbar_init(&bar_aggr[i], CWT);
                 mbar_init(&bar_carry[i], 1);
             }
             s_int[0] = 0;  // look-back failure seen by the control warp
@@ -268,10 +275,9 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 }
             };
             // A group's second tile is prepared while its first tile's look-back
-            // read is in flight: its prefixes are computed (run_pre) and, as soon
-            // as the first tile's carry is known, its inclusive value is
-            // published, so that the next group's look-back does not wait for
-            // this CTA to reach it.
+            // read is in flight: its prefixes are computed (run_pre) before the
+            // look-back resolves, so that the group's aggregate can be
+            // published first, and its carry follows from the first tile's.
             bool pre_done = false;  // the next tile's prefixes are computed (run_pre)
             Map run_pre[kV];
             for (int n = 0;; ++n) {
@@ -287,16 +293,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 // inside a group the tile before ran here: its inclusive value
                 // (y_inc) is this tile's carry
                 const bool local = (c % kGroup) != 0;
+                const int gt = (c / kGroup) * BS + rem;  // group ticket (descriptor index)
                 LookbackProbe<Map, NS> pr;
-
-                float init[NS][kV];
-#pragma unroll
-                for (int q = 0; q < NS; ++q) {
-                    F4 x{{0.f, 0.f, 0.f, 0.f}};
-                    if (c == 0 && dch < D && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
-#pragma unroll
-                    for (int j = 0; j < kV; ++j) init[q][j] = x.v[j];
-                }
                 float* car = reinterpret_cast<float*>(work_at(wb) + LY::off_carry);
                 bool ok = true;
                 Map run[kV];
@@ -307,68 +305,86 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     ok = mbar_wait_bounded(&bar_aggr[wb], uint32_t(n / kWork) & 1u, err, p.wait_ns);
                     // first look-back read, in flight while the folds are composed
                     // (issued only now, so that it sees predecessors as late as possible)
-                    if (c > 0 && !local) lookback_probe(pr, ticket - BS, p.desc, lane);
+                    if (c > 0 && !local) {
+                        if (walk) lookback_probe<Map, NS, true>(pr, gt - BS, p.desc, lane);
+                        else lookback_probe<Map, NS, false>(pr, gt - BS, p.desc, lane);
+                    }
                     prefix(wb, run);
                 }
                 float y[NS][kV];
                 if (local) {
-                    // carry = inclusive value of the group's previous tile; this
-                    // tile's inclusive value was published already if pre_done
+                    // carry = inclusive value of the group's previous tile
 #pragma unroll
                     for (int q = 0; q < NS; ++q)
 #pragma unroll
                         for (int j = 0; j < kV; ++j) y[q][j] = y_inc[q][j];
-#pragma unroll
-                    for (int j = 0; j < kV; ++j) {
-                        float x[NS], z[NS];
-#pragma unroll
-                        for (int q = 0; q < NS; ++q) x[q] = y[q][j];
-                        apply(run[j], x, z);
-#pragma unroll
-                        for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
-                    }
-                    if (!pre_done) publish_inclusive<Map, NS>(p.desc, ticket, k, y_inc, lane);
                     pre_done = false;
                 } else {
-                    // the group's next tile, if it is the next in the ring: its
+                    // the group's second tile (the next in the ring): its
                     // prefixes now, while the look-back read is in flight
-                    if (kGroup > 1) {
+                    bool two = false;
+                    if (c + 1 < p.n_chunks) {
                         const int n1 = n + 1, s1 = n1 % kStages;
                         int t1 = tk[0];
 #pragma unroll
                         for (int i = 1; i < kStages; ++i)
                             if (s1 == i) t1 = tk[i];
-                        if (t1 < p.n_tiles && t1 == ticket + BS && ((c + 1) % kGroup) != 0) {
+                        if (t1 == ticket + BS) {
                             ok = mbar_wait_bounded(&bar_aggr[n1 % kWork], uint32_t(n1 / kWork) & 1u, err, p.wait_ns) &&
                                  ok;
                             prefix(n1 % kWork, run_pre);
-                            pre_done = true;
+                            pre_done = two = true;
+                        } else {
+                            ok = false;  // the group's tiles are always issued back to back
                         }
                     }
-                    ok = lookback<Map, NS>(ticket, BS, c > 0, k, run, init, y, p.desc, lane, err, p.wait_ns, pr) && ok;
+                    if (c > 0) {
+                        // the group's aggregate (both tiles' maps composed)
+                        // goes out first, for look-backs that step over it
+                        if (walk) {
+                            Map gagg[kV];
+#pragma unroll
+                            for (int j = 0; j < kV; ++j) gagg[j] = two ? compose(run_pre[j], run[j]) : run[j];
+                            publish_aggregate<Map, NS>(p.desc, gt, k, gagg, lane);
+                            ok = lookback_resolve<Map, NS, true>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) && ok;
+                        } else {
+                            ok = lookback_resolve<Map, NS, false>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) &&
+                                 ok;
+                        }
+                    } else {
+                        // the sequence's first group: the initial state
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) {
+                            F4 x{{0.f, 0.f, 0.f, 0.f}};
+                            if (dch < D && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+#pragma unroll
+                            for (int j = 0; j < kV; ++j) y[q][j] = x.v[j];
+                        }
+                    }
+                }
+                // the state leaving this tile; at a group's head, also the
+                // state leaving the group (its inclusive value)
+#pragma unroll
+                for (int j = 0; j < kV; ++j) {
+                    float x[NS], z[NS];
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) x[q] = y[q][j];
+                    apply(run[j], x, z);
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
+                }
+                if (!local && __all_sync(0xffffffffu, ok)) {
+                    float incl[NS][kV];
 #pragma unroll
                     for (int j = 0; j < kV; ++j) {
                         float x[NS], z[NS];
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) x[q] = y[q][j];
-                        apply(run[j], x, z);
+                        for (int q = 0; q < NS; ++q) x[q] = y_inc[q][j];
+                        if (pre_done) apply(run_pre[j], x, z);
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) y_inc[q][j] = z[q];
+                        for (int q = 0; q < NS; ++q) incl[q][j] = pre_done ? z[q] : x[q];
                     }
-                    if (pre_done) {
-                        // the next tile's inclusive value, published right away
-                        float yn[NS][kV];
-#pragma unroll
-                        for (int j = 0; j < kV; ++j) {
-                            float x[NS], z[NS];
-#pragma unroll
-                            for (int q = 0; q < NS; ++q) x[q] = y_inc[q][j];
-                            apply(run_pre[j], x, z);
-#pragma unroll
-                            for (int q = 0; q < NS; ++q) yn[q][j] = z[q];
-                        }
-                        publish_inclusive<Map, NS>(p.desc, ticket + BS, k, yn, lane);
-                    }
+                    publish_inclusive<Map, NS>(p.desc, gt, k, incl, lane);
                 }
 #pragma unroll
                 for (int q = 0; q < NS; ++q) store4(car + q * kDc + lane * kV, y[q]);
@@ -391,15 +407,17 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
             }
         } else {
             // ------------------------------------------------ compute warps
-            const int ra = 2 * w, rb = 2 * w + 1;  // this warp's two steps in the tile
+            const int rp = w;             // this warp's row pair
+            const int cofs = lane * CV;   // first channel of this lane in the tile
+            const int ra = 2 * rp, rb = 2 * rp + 1;  // this warp's two steps in the tile
             int4 prev = make_int4(INT_MAX, 0, 0, 0);  // job of the previous tile
-            Jac2 Jp[2][2];  // Jacobians of the previous tile's two steps (per pair)
+            Jac2 Jp[2][NP];  // Jacobians of the previous tile's two steps (per pair)
             for (int n = 0;; ++n) {
                 const int s = n % kStages, wb = n % kWork;
                 (void)mbar_wait_bounded(&bar_full[s], uint32_t(n / kStages) & 1u, err, p.wait_ns);
                 const int4 job = s_job[s];
                 const bool valid = job.x < p.n_tiles;
-                Jac2 Jn[2][2];
+                Jac2 Jn[2][NP];
                 if (valid) {
                     // ---- sweep 1 of tile n
                     unsigned char* st = stage_at(s);
@@ -412,58 +430,60 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     float* sagg = reinterpret_cast<float*>(wk + LY::off_agg);
                     const int c = job.y, b = job.z, d0 = job.w;
                     const int l0 = c * Lc;
-                    const int dch = d0 + lane * kV;
+                    const int dch = d0 + cofs;
                     const bool chv = dch < D;
-                    float2 wv[G][2];
+                    float2 wv[G][NP];
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        F4 x = load4(sa + g * kDc + lane * kV);  // zero beyond D (TMA fill)
-                        wv[g][0] = make_float2(x.v[0], x.v[1]);
-                        wv[g][1] = make_float2(x.v[2], x.v[3]);
+                        FV<CV> x = loadv<CV>(sa + g * kDc + cofs);  // zero beyond D (TMA fill)
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) wv[g][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
                     }
                     // s^k before step a, s^k at steps a and b
-                    float2 sp[NS][2], ska[NS][2], skb[NS][2];
+                    float2 sp[NS][NP], ska[NS][NP], skb[NS][NP];
 #pragma unroll
                     for (int q = 0; q < NS; ++q) {
-                        F4 x{{0.f, 0.f, 0.f, 0.f}};
-                        if (w == 0) {
+                        FV<CV> x, xa, xb;
+#pragma unroll
+                        for (int j = 0; j < CV; ++j) x.v[j] = xa.v[j] = xb.v[j] = 0.f;
+                        if (rp == 0) {
                             if (c == 0) {
                                 const float* lin = p.s0[q];
                                 if (Seg && hdr->seg_lin[q]) lin = reinterpret_cast<const float*>(hdr->seg_lin[q]);
-                                if (chv && lin) x = load4(lin + b * D + dch);
+                                if (chv && lin) x = loadv<CV>(lin + b * D + dch);
                             } else if (!first) {
-                                x = load4(sbnd + q * kDc + lane * kV);
+                                x = loadv<CV>(sbnd + q * kDc + cofs);
                             }
                         } else if (!first) {
-                            x = load4(ss + (q * Lc + ra - 1) * kDc + lane * kV);
+                            x = loadv<CV>(ss + (q * Lc + ra - 1) * kDc + cofs);
                         }
-                        sp[q][0] = make_float2(x.v[0], x.v[1]);
-                        sp[q][1] = make_float2(x.v[2], x.v[3]);
-                        F4 xa{{0.f, 0.f, 0.f, 0.f}}, xb{{0.f, 0.f, 0.f, 0.f}};
                         if (!first) {
-                            xa = load4(ss + (q * Lc + ra) * kDc + lane * kV);
-                            xb = load4(ss + (q * Lc + rb) * kDc + lane * kV);
+                            xa = loadv<CV>(ss + (q * Lc + ra) * kDc + cofs);
+                            xb = loadv<CV>(ss + (q * Lc + rb) * kDc + cofs);
                         }
-                        ska[q][0] = make_float2(xa.v[0], xa.v[1]);
-                        ska[q][1] = make_float2(xa.v[2], xa.v[3]);
-                        skb[q][0] = make_float2(xb.v[0], xb.v[1]);
-                        skb[q][1] = make_float2(xb.v[2], xb.v[3]);
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) {
+                            sp[q][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
+                            ska[q][jp] = make_float2(xa.v[2 * jp], xa.v[2 * jp + 1]);
+                            skb[q][jp] = make_float2(xb.v[2 * jp], xb.v[2 * jp + 1]);
+                        }
                     }
-                    float2 ua[G][2], ub[G][2];
+                    float2 ua[G][NP], ub[G][NP];
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        F4 x = load4(su + (ra * G + g) * kDc + lane * kV);
-                        ua[g][0] = make_float2(x.v[0], x.v[1]);
-                        ua[g][1] = make_float2(x.v[2], x.v[3]);
-                        F4 z = load4(su + (rb * G + g) * kDc + lane * kV);
-                        ub[g][0] = make_float2(z.v[0], z.v[1]);
-                        ub[g][1] = make_float2(z.v[2], z.v[3]);
+                        FV<CV> x = loadv<CV>(su + (ra * G + g) * kDc + cofs);
+                        FV<CV> z = loadv<CV>(su + (rb * G + g) * kDc + cofs);
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) {
+                            ua[g][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
+                            ub[g][jp] = make_float2(z.v[2 * jp], z.v[2 * jp + 1]);
+                        }
                     }
                     const bool va = (l0 + ra) < L && chv, vb = (l0 + rb) < L && chv;
-                    Map2 agg2[2];
-                    float2 offa[NS][2], offb[NS][2];
+                    Map2 agg2[NP];
+                    float2 offa[NS][NP], offb[NS][NP];
 #pragma unroll
-                    for (int jp = 0; jp < 2; ++jp) {
+                    for (int jp = 0; jp < NP; ++jp) {
                         float2 s_a[NS], s_b[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS], ja[NS], jb[NS];
 #pragma unroll
                         for (int q = 0; q < NS; ++q) {
@@ -505,19 +525,27 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     }
 #pragma unroll
                     for (int q = 0; q < NS; ++q) {
-                        float va4[kV] = {offa[q][0].x, offa[q][0].y, offa[q][1].x, offa[q][1].y};
-                        float vb4[kV] = {offb[q][0].x, offb[q][0].y, offb[q][1].x, offb[q][1].y};
-                        store4(ss + (q * Lc + ra) * kDc + lane * kV, va4);  // step a's state is no longer read
-                        store4(slast + (q * CW + w) * kDc + lane * kV, vb4);  // step b's state is the next warp's input
+                        float va4[CV], vb4[CV];
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) {
+                            va4[2 * jp] = offa[q][jp].x;
+                            va4[2 * jp + 1] = offa[q][jp].y;
+                            vb4[2 * jp] = offb[q][jp].x;
+                            vb4[2 * jp + 1] = offb[q][jp].y;
+                        }
+                        storev<CV>(ss + (q * Lc + ra) * kDc + cofs, va4);   // step a's state is no longer read
+                        storev<CV>(slast + (q * CW + rp) * kDc + cofs, vb4);  // step b's state is the next pair's input
                     }
                     {
-                        Map a1[kV] = {agg2[0].lane(0), agg2[0].lane(1), agg2[1].lane(0), agg2[1].lane(1)};
 #pragma unroll
                         for (int i = 0; i < NC; ++i) {
-                            float v4[kV];
+                            float v4[CV];
 #pragma unroll
-                            for (int j = 0; j < kV; ++j) v4[j] = a1[j].get(i);
-                            store4(sagg + (i * CW + w) * kDc + lane * kV, v4);
+                            for (int jp = 0; jp < NP; ++jp) {
+                                v4[2 * jp] = agg2[jp].lane(0).get(i);
+                                v4[2 * jp + 1] = agg2[jp].lane(1).get(i);
+                            }
+                            storev<CV>(sagg + (i * CW + rp) * kDc + cofs, v4);
                         }
                     }
                     __syncwarp();
@@ -537,34 +565,34 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     const float* car = reinterpret_cast<const float*>(wk + LY::off_carry);
                     const int c = prev.y, b = prev.z, d0 = prev.w;
                     const int l0 = c * Lc;
-                    const int dch = d0 + lane * kV;
+                    const int dch = d0 + cofs;
                     const bool chv = dch < D && !s_int[0];
-                    float2 wv[G][2];
+                    float2 wv[G][NP];
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        F4 x = load4(sa + g * kDc + lane * kV);
-                        wv[g][0] = make_float2(x.v[0], x.v[1]);
-                        wv[g][1] = make_float2(x.v[2], x.v[3]);
+                        FV<CV> x = loadv<CV>(sa + g * kDc + cofs);
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) wv[g][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
                     }
                     // state entering this warp's steps = its prefix map applied to the tile's carry
-                    float2 y0[NS][2];
+                    float2 y0[NS][NP];
                     {
-                        Map2 pre[2];
+                        Map2 pre[NP];
 #pragma unroll
                         for (int i = 0; i < NC; ++i) {
-                            F4 v = load4(spre + (i * CW + w) * kDc + lane * kV);
-                            pre[0].set(i, make_float2(v.v[0], v.v[1]));
-                            pre[1].set(i, make_float2(v.v[2], v.v[3]));
+                            FV<CV> v = loadv<CV>(spre + (i * CW + rp) * kDc + cofs);
+#pragma unroll
+                            for (int jp = 0; jp < NP; ++jp) pre[jp].set(i, make_float2(v.v[2 * jp], v.v[2 * jp + 1]));
                         }
-                        float2 ct[NS][2];
+                        float2 ct[NS][NP];
 #pragma unroll
                         for (int q = 0; q < NS; ++q) {
-                            F4 x = load4(car + q * kDc + lane * kV);
-                            ct[q][0] = make_float2(x.v[0], x.v[1]);
-                            ct[q][1] = make_float2(x.v[2], x.v[3]);
+                            FV<CV> x = loadv<CV>(car + q * kDc + cofs);
+#pragma unroll
+                            for (int jp = 0; jp < NP; ++jp) ct[q][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
                         }
 #pragma unroll
-                        for (int jp = 0; jp < 2; ++jp) {
+                        for (int jp = 0; jp < NP; ++jp) {
                             float2 x[NS], z[NS];
 #pragma unroll
                             for (int q = 0; q < NS; ++q) x[q] = ct[q][jp];
@@ -573,30 +601,32 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             for (int q = 0; q < NS; ++q) y0[q][jp] = z[q];
                         }
                     }
-                    float2 offa[NS][2], offb[NS][2], ua[G][2], ub[G][2];
+                    float2 offa[NS][NP], offb[NS][NP], ua[G][NP], ub[G][NP];
 #pragma unroll
                     for (int q = 0; q < NS; ++q) {
-                        F4 xa = load4(ss + (q * Lc + ra) * kDc + lane * kV);
-                        F4 xb = load4(slast + (q * CW + w) * kDc + lane * kV);
-                        offa[q][0] = make_float2(xa.v[0], xa.v[1]);
-                        offa[q][1] = make_float2(xa.v[2], xa.v[3]);
-                        offb[q][0] = make_float2(xb.v[0], xb.v[1]);
-                        offb[q][1] = make_float2(xb.v[2], xb.v[3]);
+                        FV<CV> xa = loadv<CV>(ss + (q * Lc + ra) * kDc + cofs);
+                        FV<CV> xb = loadv<CV>(slast + (q * CW + rp) * kDc + cofs);
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) {
+                            offa[q][jp] = make_float2(xa.v[2 * jp], xa.v[2 * jp + 1]);
+                            offb[q][jp] = make_float2(xb.v[2 * jp], xb.v[2 * jp + 1]);
+                        }
                     }
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        F4 x = load4(su + (ra * G + g) * kDc + lane * kV);
-                        ua[g][0] = make_float2(x.v[0], x.v[1]);
-                        ua[g][1] = make_float2(x.v[2], x.v[3]);
-                        F4 z = load4(su + (rb * G + g) * kDc + lane * kV);
-                        ub[g][0] = make_float2(z.v[0], z.v[1]);
-                        ub[g][1] = make_float2(z.v[2], z.v[3]);
+                        FV<CV> x = loadv<CV>(su + (ra * G + g) * kDc + cofs);
+                        FV<CV> z = loadv<CV>(su + (rb * G + g) * kDc + cofs);
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) {
+                            ua[g][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
+                            ub[g][jp] = make_float2(z.v[2 * jp], z.v[2 * jp + 1]);
+                        }
                     }
                     const long long la = l0 + ra, lb = l0 + rb;
                     const bool va = la < L && chv, vb = lb < L && chv;
-                    float2 ya[NS][2], yb[NS][2];
+                    float2 ya[NS][NP], yb[NS][NP];
 #pragma unroll
-                    for (int jp = 0; jp < 2; ++jp) {
+                    for (int jp = 0; jp < NP; ++jp) {
                         float2 s0v[NS], sav[NS], sbv[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS], t0[NS], t1[NS];
 #pragma unroll
                         for (int q = 0; q < NS; ++q) s0v[q] = y0[q][jp];
@@ -625,20 +655,20 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     }
 #pragma unroll
                     for (int q = 0; q < NS; ++q) {
-                        if (va)
-                            __stcg(reinterpret_cast<float4*>(p.st[q] + ((b * L + la) * D + dch)),
-                                   make_float4(ya[q][0].x, ya[q][0].y, ya[q][1].x, ya[q][1].y));
-                        if (vb)
-                            __stcg(reinterpret_cast<float4*>(p.st[q] + ((b * L + lb) * D + dch)),
-                                   make_float4(yb[q][0].x, yb[q][0].y, yb[q][1].x, yb[q][1].y));
-                    }
-                    if (w == CW - 1 && c + 1 < p.n_chunks && chv) {
+                        float oa4[CV], ob4[CV];
 #pragma unroll
-                        for (int q = 0; q < NS; ++q)
-                            __stcg(reinterpret_cast<float4*>(
-                                       p.bnd + ((((size_t)((k + 1) & 1) * NS + q) * p.B + b) * p.n_chunks + c) *
-                                                   Dpad + dch),
-                                   make_float4(yb[q][0].x, yb[q][0].y, yb[q][1].x, yb[q][1].y));
+                        for (int jp = 0; jp < NP; ++jp) {
+                            oa4[2 * jp] = ya[q][jp].x;
+                            oa4[2 * jp + 1] = ya[q][jp].y;
+                            ob4[2 * jp] = yb[q][jp].x;
+                            ob4[2 * jp + 1] = yb[q][jp].y;
+                        }
+                        if (va) stcgv<CV>(p.st[q] + ((b * L + la) * D + dch), oa4);
+                        if (vb) stcgv<CV>(p.st[q] + ((b * L + lb) * D + dch), ob4);
+                        if (rp == CW - 1 && c + 1 < p.n_chunks && chv)
+                            stcgv<CV>(p.bnd + ((((size_t)((k + 1) & 1) * NS + q) * p.B + b) * p.n_chunks + c) * Dpad +
+                                          dch,
+                                      ob4);
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bar_empty[sp_]);
@@ -648,7 +678,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 #pragma unroll
                 for (int r = 0; r < 2; ++r)
 #pragma unroll
-                    for (int jp = 0; jp < 2; ++jp) Jp[r][jp] = Jn[r][jp];
+                    for (int jp = 0; jp < NP; ++jp) Jp[r][jp] = Jn[r][jp];
             }
         }
 
@@ -660,14 +690,14 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
         }
         if (lane == 0) {
             s_red[w] = rpost;
-            s_red[CW + 1 + w] = rpre;
+            s_red[CWT + 1 + w] = rpre;
         }
         __syncthreads();
         if (tid == 0) {
             float a = 0.f, b2 = 0.f;
-            for (int i = 0; i <= CW; ++i) {
+            for (int i = 0; i <= CWT; ++i) {
                 a = max_keep_nan(a, s_red[i]);
-                b2 = max_keep_nan(b2, s_red[CW + 1 + i]);
+                b2 = max_keep_nan(b2, s_red[CWT + 1 + i]);
             }
             // non-negative floats (and NaN) order like their bit patterns
             atomicMax(&hdr->res[slot], __float_as_uint(a) & 0x7fffffffu);

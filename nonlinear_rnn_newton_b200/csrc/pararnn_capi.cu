@@ -67,7 +67,7 @@ constexpr size_t kSelftestWorkspace = 16384;
 #ifndef PARARNN_WS_LSTM_WARPS
 #define PARARNN_WS_LSTM_WARPS 7
 #endif
-// compute warps per CTA (two steps each); fp32 gates need twice the staging
+// row pairs per tile (two steps each); fp32 gates need twice the staging
 // space, so their tiles are half as long
 template <class UT> constexpr int gru_tile_arg() { return sizeof(UT) == 2 ? PARARNN_WS_GRU_WARPS : PARARNN_WS_GRU_WARPS / 2; }
 template <class UT> constexpr int lstm_tile_arg() { return sizeof(UT) == 2 ? PARARNN_WS_LSTM_WARPS : PARARNN_WS_LSTM_WARPS / 2; }
@@ -112,16 +112,32 @@ struct ScanLayout {
     size_t desc, extra, total;
 };
 
-// header | tile descriptors (tagged 64-bit words) | extra (boundary / partial
-// sums).  Header and descriptors are zeroed before every launch.
-ScanLayout scan_layout(const Shape& s, int desc_words, size_t extra_bytes)
+// header | look-back descriptors (tagged 64-bit words; one per tile, or
+// n_desc of them) | extra (boundary / partial sums).  Header and descriptors
+// are zeroed before every launch.
+ScanLayout scan_layout(const Shape& s, int desc_words, size_t extra_bytes, long long n_desc = -1)
 {
     ScanLayout ly;
     ly.desc = sizeof(WsHeader);
-    ly.extra = align256(ly.desc + size_t(s.n_tiles) * desc_words * 8);
+    ly.extra = align256(ly.desc + size_t(n_desc < 0 ? s.n_tiles : n_desc) * desc_words * 8);
     ly.total = align256(ly.extra + extra_bytes);
     return ly;
 }
+
+// the fused solve keeps one look-back descriptor per group of chunks
+long long solve_descs(const Shape& s) { return solve_desc_count(s.n_chunks, s.B * s.S); }
+
+// Whether the solve's look-backs step back over predecessors' aggregates.
+// Every CTA holds about two groups, so grid / sequences groups of one
+// sequence are in flight.  With few of them (many sequences) a group's
+// predecessor publishes its inclusive value about as soon as a step back
+// would find anything, and waiting for it -- with no aggregates published or
+// read at all -- is faster (measured: ParaLSTM B=8 L=4096 D=1024 1.32 ms
+// against 1.97 ms stepping back; ParaGRU 0.620 against 0.646 ms); with many
+// (one sequence of 2048 channels: 16 slabs over 148 CTAs) a chain of
+// inclusive values paces the pass and stepping back is faster (ParaGRU B=1
+// L=65536 D=2048: 2.81 against 3.17 ms).
+int solve_lookback_walks(int grid, long long sequences) { return grid >= 4 * sequences ? 1 : 0; }
 
 size_t solve_bnd_bytes(const Shape& s, int NS)
 {
@@ -268,19 +284,19 @@ pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid, int th
 
 // in: where the first pass reads the states (segment passes: the given
 // iterate; NULL = st); slin, warm: see NewtonParams.
-template <class Cell, class UT, int T, bool Seg = false>
-pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
-                             float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream,
-                             const float* const* in = nullptr, const float* const* slin = nullptr, int warm = 0)
+template <class Cell, class UT, int T, bool Seg, int LB>
+pararnn_status launch_newton_k(const Shape& s, const void* u, pararnn_dtype dt, const float* a,
+                               const float* const s0[2], float* const st[2], float tol, int max_iters, void* ws,
+                               cudaStream_t stream, const float* const* in, const float* const* slin, int warm)
 {
     constexpr int NS = Cell::NS;
     constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
     using KL = NewtonWsLayout<Cell, UT, T>;  // T = compute warps (two steps each)
-    auto kern = newton_solve_ws_kernel<Cell, UT, T, Seg>;
+    auto kern = newton_solve_ws_kernel<Cell, UT, T, Seg, LB>;
     constexpr int threads = KL::threads;
     // the TMA boxes must be exactly the kernel's tile
     if (s.Lc != KL::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, KL::Lc);
-    const ScanLayout ly = scan_layout(s, desc_words, solve_bnd_bytes(s, NS));
+    const ScanLayout ly = scan_layout(s, desc_words, solve_bnd_bytes(s, NS), solve_descs(s));
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));  // header + descriptors
 
@@ -328,6 +344,7 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
 
     int grid = 0;
     TRY(resident_grid(kern, KL::smem_bytes, s.n_tiles, &grid, threads));
+    p.lb_walk = LB;
     CUtensorMap ta, tb;
     TRY(map_weights(&ta, a, Cell::G, s));
     TRY(map_bnd(&tb, p.bnd, NS, s));
@@ -336,6 +353,21 @@ pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, co
                                          KL::smem_bytes, stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return PARARNN_OK;
+}
+
+// The fused solve in the look-back mode that suits the shape (see
+// solve_lookback_walks): stepping back over aggregates, or waiting for
+// inclusive values.  Both kernel variants run one CTA per SM.
+template <class Cell, class UT, int T, bool Seg = false>
+pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
+                             float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream,
+                             const float* const* in = nullptr, const float* const* slin = nullptr, int warm = 0)
+{
+    int sms = 0;
+    TRY(device_info(&sms));
+    if (solve_lookback_walks(std::min(s.n_tiles, sms), s.B * s.S))
+        return launch_newton_k<Cell, UT, T, Seg, 1>(s, u, dt, a, s0, st, tol, max_iters, ws, stream, in, slin, warm);
+    return launch_newton_k<Cell, UT, T, Seg, 0>(s, u, dt, a, s0, st, tol, max_iters, ws, stream, in, slin, warm);
 }
 
 size_t solve_ws_bytes(int cell, long long B, long long L, long long D)
@@ -347,8 +379,8 @@ size_t solve_ws_bytes(int cell, long long B, long long L, long long D)
     pararnn_status st = make_shape(B, L, D, cell == 0 ? kLcGru : kLcLstm, &s);
     memcpy(t_err, saved, sizeof(t_err));
     if (st != PARARNN_OK) return 0;
-    if (cell == 0) return scan_layout(s, TileDesc<Aff<1>, 1>::words, solve_bnd_bytes(s, 1)).total;
-    return scan_layout(s, TileDesc<Aff<2>, 2>::words, solve_bnd_bytes(s, 2)).total;
+    if (cell == 0) return scan_layout(s, TileDesc<Aff<1>, 1>::words, solve_bnd_bytes(s, 1), solve_descs(s)).total;
+    return scan_layout(s, TileDesc<Aff<2>, 2>::words, solve_bnd_bytes(s, 2), solve_descs(s)).total;
 }
 
 // Host-side argument checks of a solve (everything but the workspace); no

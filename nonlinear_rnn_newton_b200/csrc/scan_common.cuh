@@ -167,126 +167,35 @@ struct LookbackProbe {
     unsigned long long wa[kV * Map::kFloats];
 };
 
-template <class Map, int NS>
+// (WithAgg = false: the inclusive value only, for a look-back that waits for
+// it instead of stepping back.)
+template <class Map, int NS, bool WithAgg = true>
 __device__ __forceinline__ void lookback_probe(LookbackProbe<Map, NS>& pr, int pred_ticket,
                                                const unsigned long long* desc, int lane)
 {
     using TD = TileDesc<Map, NS>;
     const unsigned long long* pd = desc + (size_t)pred_ticket * TD::words;
     load_words(pd + TD::agg_words + lane * kV * NS, pr.wi);
-    load_words(pd + lane * kV * Map::kFloats, pr.wa);
+    if (WithAgg) load_words(pd + lane * kV * Map::kFloats, pr.wa);
 }
 
-// Decoupled look-back, run by one full warp; lane owns channels lane*kV..+kV-1.
-//   ticket:    this tile's ticket; its predecessor is ticket - stride
-//   has_pred:  false for the first tile of a sequence (carry = `init`)
-//   epoch:     tags 2*epoch+1 (aggregate), 2*epoch+2 (inclusive)
-//   ta:        this tile's aggregate maps
-//   carry:     out: value entering this tile (the predecessors' inclusive)
-//   pr:        the first probe (lookback_probe of ticket - stride), if has_pred
-// Publishes the aggregate (if there is a predecessor) and, once the carry is
-// known, the inclusive value apply(ta, carry).  Each step back reads the
-// predecessor's inclusive value and aggregate together (one round trip).
-// Each lane walks back on its own; a wait that runs out of time raises
-// PARARNN_ERR_TIMEOUT and returns false.
+// Publish maps (a tile's or a group's aggregate) under tag 2*epoch+1.
 template <class Map, int NS>
-__device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, int epoch, const Map (&ta)[kV],
-                                         const float (&init)[NS][kV], float (&carry)[NS][kV],
-                                         unsigned long long* desc, int lane, int* err,
-                                         unsigned long long wait_ns, LookbackProbe<Map, NS>& pr)
+__device__ __forceinline__ void publish_aggregate(unsigned long long* desc, int ticket, int epoch, const Map (&ta)[kV],
+                                                  int lane)
 {
     using TD = TileDesc<Map, NS>;
     constexpr int NC = Map::kFloats;
-    const unsigned t_agg = 2u * epoch + 1u, t_incl = 2u * epoch + 2u;
-    unsigned long long* mine = desc + (size_t)ticket * TD::words;
+    float av[kV * NC];
 #pragma unroll
-    for (int q = 0; q < NS; ++q)
+    for (int j = 0; j < kV; ++j)
 #pragma unroll
-        for (int j = 0; j < kV; ++j) carry[q][j] = init[q][j];
-    bool ok = true;
-    if (has_pred) {
-        {
-            float av[kV * NC];
-#pragma unroll
-            for (int j = 0; j < kV; ++j)
-#pragma unroll
-                for (int i = 0; i < NC; ++i) av[j * NC + i] = ta[j].get(i);
-            publish_words(mine + lane * kV * NC, av, t_agg);
-        }
-        Map acc[kV];
-#pragma unroll
-        for (int j = 0; j < kV; ++j) acc[j] = Map::identity();
-        int jt = ticket - stride;
-        bool done = false;
-        uint64_t t0 = 0;
-        unsigned spins = 0;
-        while (__any_sync(0xffffffffu, !done)) {
-            if (!done) {
-                float iv[kV * NS];
-                float av[kV * NC];
-                if (unpack_words(pr.wi, iv, t_incl)) {
-#pragma unroll
-                    for (int j = 0; j < kV; ++j) {
-                        float x[NS], y[NS];
-#pragma unroll
-                        for (int q = 0; q < NS; ++q) x[q] = iv[j * NS + q];
-                        apply(acc[j], x, y);
-#pragma unroll
-                        for (int q = 0; q < NS; ++q) carry[q][j] = y[q];
-                    }
-                    done = true;
-                } else if (unpack_words(pr.wa, av, t_agg)) {
-#pragma unroll
-                    for (int j = 0; j < kV; ++j) {
-                        Map e;
-#pragma unroll
-                        for (int i = 0; i < NC; ++i) e.set(i, av[j * NC + i]);
-                        acc[j] = compose(acc[j], e);
-                    }
-                    jt -= stride;
-                    spins = 0;
-                    lookback_probe(pr, jt, desc, lane);
-                } else {
-                    // predecessor not published yet: back off, bounded
-                    if ((++spins & 15u) == 0u) {
-                        if (error_raised(err)) {
-                            ok = false;
-                            done = true;
-                        } else {
-                            const uint64_t now = global_timer_ns();
-                            if (t0 == 0) {
-                                t0 = now;
-                            } else if (now - t0 > wait_ns) {
-                                raise_error(err, PARARNN_ERR_TIMEOUT);
-                                ok = false;
-                                done = true;
-                            }
-                        }
-                    }
-                    if (spins > 32) __nanosleep(64);
-                    if (!done) lookback_probe(pr, jt, desc, lane);
-                }
-            }
-        }
-    }
-    if (ok) {
-        float iv[kV * NS];
-#pragma unroll
-        for (int j = 0; j < kV; ++j) {
-            float x[NS], y[NS];
-#pragma unroll
-            for (int q = 0; q < NS; ++q) x[q] = carry[q][j];
-            apply(ta[j], x, y);
-#pragma unroll
-            for (int q = 0; q < NS; ++q) iv[j * NS + q] = y[q];
-        }
-        publish_words(mine + TD::agg_words + lane * kV * NS, iv, t_incl);
-    }
-    return __all_sync(0xffffffffu, ok);
+        for (int i = 0; i < NC; ++i) av[j * NC + i] = ta[j].get(i);
+    publish_words(desc + (size_t)ticket * TD::words + lane * kV * NC, av, 2u * epoch + 1u);
 }
 
-// Publish a tile's inclusive value when its carry is known without a
-// look-back (the tile before ran in the same CTA).
+// Publish an inclusive value (the state leaving a tile or group) under tag
+// 2*epoch+2.
 template <class Map, int NS>
 __device__ __forceinline__ void publish_inclusive(unsigned long long* desc, int ticket, int epoch,
                                                   const float (&incl)[NS][kV], int lane)
@@ -298,6 +207,123 @@ __device__ __forceinline__ void publish_inclusive(unsigned long long* desc, int 
 #pragma unroll
         for (int q = 0; q < NS; ++q) iv[j * NS + q] = incl[q][j];
     publish_words(desc + (size_t)ticket * TD::words + TD::agg_words + lane * kV * NS, iv, 2u * epoch + 2u);
+}
+
+// Decoupled look-back, run by one full warp; lane owns channels lane*kV..+kV-1.
+// Resolves the value entering tile `ticket` (whose predecessor is
+// ticket - stride) from its predecessors' descriptors:
+//   epoch:     tags 2*epoch+1 (aggregate), 2*epoch+2 (inclusive)
+//   carry:     out: value entering this tile (the predecessors' inclusive)
+//   pr:        the first probe (lookback_probe of ticket - stride)
+//   Walk:      step back over a predecessor that has published only its
+//              aggregate (the decoupled look-back); if false, wait for the
+//              predecessor's inclusive value instead (a chain of inclusive
+//              values, which is faster when few tiles of one sequence are in
+//              flight at once) and read no aggregates at all (the probe must
+//              then come from lookback_probe<..., false>)
+// Each step back reads the predecessor's inclusive value and aggregate
+// together (one round trip).  Each lane walks back on its own; a wait that
+// runs out of time raises PARARNN_ERR_TIMEOUT and returns false.
+template <class Map, int NS, bool Walk = true>
+__device__ __forceinline__ bool lookback_resolve(int ticket, int stride, int epoch, float (&carry)[NS][kV],
+                                                 const unsigned long long* desc, int lane, int* err,
+                                                 unsigned long long wait_ns, LookbackProbe<Map, NS>& pr)
+{
+    constexpr int NC = Map::kFloats;
+    const unsigned t_agg = 2u * epoch + 1u, t_incl = 2u * epoch + 2u;
+    bool ok = true;
+    Map acc[kV];
+#pragma unroll
+    for (int j = 0; j < kV; ++j) acc[j] = Map::identity();
+    int jt = ticket - stride;
+    bool done = false;
+    uint64_t t0 = 0;
+    unsigned spins = 0;
+    while (__any_sync(0xffffffffu, !done)) {
+        if (!done) {
+            float iv[kV * NS];
+            float av[kV * NC];
+            if (unpack_words(pr.wi, iv, t_incl)) {
+#pragma unroll
+                for (int j = 0; j < kV; ++j) {
+                    float x[NS], y[NS];
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) x[q] = iv[j * NS + q];
+                    apply(acc[j], x, y);
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) carry[q][j] = y[q];
+                }
+                done = true;
+            } else if (Walk && unpack_words(pr.wa, av, t_agg)) {
+#pragma unroll
+                for (int j = 0; j < kV; ++j) {
+                    Map e;
+#pragma unroll
+                    for (int i = 0; i < NC; ++i) e.set(i, av[j * NC + i]);
+                    acc[j] = compose(acc[j], e);
+                }
+                jt -= stride;
+                spins = 0;
+                lookback_probe(pr, jt, desc, lane);
+            } else {
+                // predecessor not published yet: back off, bounded
+                if ((++spins & 15u) == 0u) {
+                    if (error_raised(err)) {
+                        ok = false;
+                        done = true;
+                    } else {
+                        const uint64_t now = global_timer_ns();
+                        if (t0 == 0) {
+                            t0 = now;
+                        } else if (now - t0 > wait_ns) {
+                            raise_error(err, PARARNN_ERR_TIMEOUT);
+                            ok = false;
+                            done = true;
+                        }
+                    }
+                }
+                if (spins > 32) __nanosleep(64);
+                if (!done) lookback_probe<Map, NS, Walk>(pr, jt, desc, lane);
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Decoupled look-back of one tile with aggregate `ta`: publishes the
+// aggregate (if there is a predecessor), resolves the carry (`init` for the
+// first tile of a sequence) and publishes the inclusive value
+// apply(ta, carry).  False if a wait gave up.
+template <class Map, int NS>
+__device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, int epoch, const Map (&ta)[kV],
+                                         const float (&init)[NS][kV], float (&carry)[NS][kV],
+                                         unsigned long long* desc, int lane, int* err,
+                                         unsigned long long wait_ns, LookbackProbe<Map, NS>& pr)
+{
+    bool ok = true;
+    if (has_pred) {
+        publish_aggregate<Map, NS>(desc, ticket, epoch, ta, lane);
+        ok = lookback_resolve<Map, NS, true>(ticket, stride, epoch, carry, desc, lane, err, wait_ns, pr);
+    } else {
+#pragma unroll
+        for (int q = 0; q < NS; ++q)
+#pragma unroll
+            for (int j = 0; j < kV; ++j) carry[q][j] = init[q][j];
+    }
+    if (ok) {
+        float incl[NS][kV];
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+            float x[NS], y[NS];
+#pragma unroll
+            for (int q = 0; q < NS; ++q) x[q] = carry[q][j];
+            apply(ta[j], x, y);
+#pragma unroll
+            for (int q = 0; q < NS; ++q) incl[q][j] = y[q];
+        }
+        publish_inclusive<Map, NS>(desc, ticket, epoch, incl, lane);
+    }
+    return ok;
 }
 
 // Look-back without an early probe.
