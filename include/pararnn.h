@@ -149,6 +149,13 @@ PARARNN_API pararnn_status pararnn_lstm_solve_async(const void* u, pararnn_dtype
                                         int max_iters, void* workspace, size_t workspace_bytes,
                                         pararnn_stream_t stream);
 
+/* Queues on `stream` a copy of the last solve's (or segment pass's) residual
+ * into out[0] and 1.0f into out[1] if a device-side error was raised (else
+ * 0.0f); out is two device floats.  Asynchronous: for host loops that reduce
+ * the outcome across GPUs before reading it. */
+PARARNN_API pararnn_status pararnn_result_to_device(const void* workspace, float* out,
+                                                    pararnn_stream_t stream);
+
 /* Synchronises `stream` and reads the outcome of the last solve or adjoint
  * queued on `workspace`.  Returns result->status (or an error if the read
  * itself fails).  `result` is a host pointer. */
@@ -327,18 +334,23 @@ PARARNN_API pararnn_status pararnn_read_pass_times(const void* workspace, pararn
 /* ------------------------------------------------- segments of a sequence */
 
 /* The Newton solve with the sequence split into segments, one per GPU ("A
- * sacada: método de Newton": every iteration solves a linear recurrence;
- * over a segment its solution is affine in the state entering the
- * segment).  One iteration k -> k+1 on each segment:
- *   1. pararnn_*_segment_pass with s_carry = 0 (beta), then once per state
- *      component j with s_carry = e_j (unit j), each from the same iterate;
- *   2. gather the passes' last-step states of every segment, in segment
- *      order, into ends [R][1 + NS][NS][B][D] (the exchange between GPUs);
- *   3. pararnn_segment_carries -> the state entering every segment;
- *   4. pararnn_*_segment_update with this segment's carry -> the iterate
- *      k+1 and its residual; the maximum over segments decides.
- * The iterate entering a segment at k+1 is its carry, which is also the
- * state the next pass linearises the segment's first step at.
+ * sacada: método de Newton": every iteration solves a linear recurrence
+ * whose step maps s -> J_l s + o_l depend only on the iterate H^k, so over a
+ * segment they compose into one affine map of the state entering it).  One
+ * iteration k on each segment:
+ *   1. pararnn_*_segment_fold: the segment's record from H^k -- its step
+ *      maps folded (steps 2..Ls), the iterate's first and last states, the
+ *      first step's gates, the residual over steps 2..Ls;
+ *   2. gather every segment's record, in segment order (the one data
+ *      exchange between GPUs: pararnn_segment_record_floats each);
+ *   3. pararnn_*_segment_combine: the records composed in order -> the new
+ *      state entering this segment (carry), the iterate's state before it
+ *      (lin), and max |F(H^k)| over all segments, the same on every GPU;
+ *      stop here if it is <= tol (or k = max_iters);
+ *   4. pararnn_*_segment_pass(s_in = H^k, s_lin = lin, s_carry = carry,
+ *      s_out = H^k in place) -> H^{k+1} on the segment; its residual (read
+ *      with pararnn_read_result) maxed over the segments is that of H^{k+1},
+ *      which takes the next decision without another fold.
  * Components are stacked one after another: [NS][B][Ls][D] for states over
  * the segment, [NS][B][D] for one step (LSTM: c, then h).  Device pointers,
  * 16-byte aligned, D a multiple of 8; all calls asynchronous on `stream`.
@@ -346,9 +358,11 @@ PARARNN_API pararnn_status pararnn_read_pass_times(const void* workspace, pararn
  * segment_pass: one pass over the segment (gates u [B][Ls][G][D] of its
  * steps) from the iterate s_in (NULL = the zero guess H^0), linearising the
  * first step at s_lin (the iterate's state before the segment; NULL = 0),
- * with s_carry (NULL = 0) as the new state before it.  Writes s_out (must not
- * overlap s_in) and, if s_end is not NULL, the last step's states.  The
- * workspace is the solve's (pararnn_*_workspace_size(B, Ls, D)). */
+ * with s_carry (NULL = 0) as the new state before it.  Writes s_out (s_in
+ * itself, or a buffer that does not overlap it) and, if s_end is not NULL,
+ * the last step's states.  The workspace is the solve's
+ * (pararnn_*_workspace_size(B, Ls, D)); its result (pararnn_read_result)
+ * holds the residual of s_out with s_carry as the state before it. */
 PARARNN_API pararnn_status pararnn_gru_segment_pass(const void* u, pararnn_dtype u_dtype,
                                                     const float* a, const float* h_in,
                                                     const float* h_lin, const float* h_carry,
@@ -363,29 +377,43 @@ PARARNN_API pararnn_status pararnn_lstm_segment_pass(const void* u, pararnn_dtyp
                                                      int64_t L, int64_t D, void* workspace,
                                                      size_t workspace_bytes,
                                                      pararnn_stream_t stream);
-/* segment_update: s_out = beta + sum_j (unit_j - beta) carry_j, with beta
- * [NS][B][Ls][D], unit [NS][NS][B][Ls][D] (pass j, then component), carry
- * [NS][B][D]; and max |s_l - f(s_{l-1}, u_l)| over the segment (s_{-1} =
- * carry) combined into *residual, a device float the caller sets to 0 first
- * (a maximum over launches; NaN kept). */
-PARARNN_API pararnn_status pararnn_gru_segment_update(const void* u, pararnn_dtype u_dtype,
-                                                      const float* a, const float* beta,
-                                                      const float* unit, const float* carry,
-                                                      float* h_out, float* residual, int64_t B,
-                                                      int64_t L, int64_t D,
-                                                      pararnn_stream_t stream);
-PARARNN_API pararnn_status pararnn_lstm_segment_update(const void* u, pararnn_dtype u_dtype,
-                                                       const float* a, const float* beta,
-                                                       const float* unit, const float* carry,
-                                                       float* s_out, float* residual, int64_t B,
-                                                       int64_t L, int64_t D,
-                                                       pararnn_stream_t stream);
-/* segment_carries: from ends [R][1 + NS][NS][B][D] and the initial state s0
- * [NS][B][D] (NULL = 0), the state entering every segment, carries
- * [R][NS][B][D]: c_0 = s0, c_{r+1} = beta_r + sum_j (unit_rj - beta_r) c_r[j]. */
-PARARNN_API pararnn_status pararnn_segment_carries(const float* ends, const float* s0,
-                                                   float* carries, int n_segments, int n_state,
-                                                   int64_t B, int64_t D, pararnn_stream_t stream);
+/* Floats of one segment's record (n_state = 1: ParaGRU, 2: ParaLSTM) for B x
+ * D channels: F = NC + 2 NS + G fields of B*D floats (NC = 2 or 6 map
+ * entries, NS = 1 or 2, G = 3 or 4), then 4 floats (the first is the
+ * residual over the segment's steps 2..Ls).  0 for invalid arguments. */
+PARARNN_API size_t pararnn_segment_record_floats(int n_state, int64_t B, int64_t D);
+/* Workspace bytes of segment_fold (its per-128-step partial folds). */
+PARARNN_API size_t pararnn_segment_fold_workspace_size(int n_state, int64_t B, int64_t L, int64_t D);
+/* segment_fold: the segment's record (overwritten in full) from the iterate
+ * s_in [NS][B][Ls][D] (NULL = the zero guess) and the gates u [B][Ls][G][D]
+ * (bf16 or fp32). */
+PARARNN_API pararnn_status pararnn_gru_segment_fold(const void* u, pararnn_dtype u_dtype,
+                                                    const float* a, const float* h_in,
+                                                    float* record, int64_t B, int64_t L,
+                                                    int64_t D, void* workspace,
+                                                    size_t workspace_bytes,
+                                                    pararnn_stream_t stream);
+PARARNN_API pararnn_status pararnn_lstm_segment_fold(const void* u, pararnn_dtype u_dtype,
+                                                     const float* a, const float* s_in,
+                                                     float* record, int64_t B, int64_t L,
+                                                     int64_t D, void* workspace,
+                                                     size_t workspace_bytes,
+                                                     pararnn_stream_t stream);
+/* segment_combine: records [n_segments][record_floats] in segment order and
+ * the initial state s0 [NS][B][D] (NULL = 0) -> for segment `index`: carry
+ * (the state entering it at iterate k+1) and lin (the iterate's state before
+ * it), [NS][B][D]; *residual (a device float, overwritten) = max |F(H^k)|
+ * over every segment's steps, NaN kept. */
+PARARNN_API pararnn_status pararnn_gru_segment_combine(const float* records, int n_segments,
+                                                       int index, const float* a,
+                                                       const float* h0, float* h_carry,
+                                                       float* h_lin, float* residual, int64_t B,
+                                                       int64_t D, pararnn_stream_t stream);
+PARARNN_API pararnn_status pararnn_lstm_segment_combine(const float* records, int n_segments,
+                                                        int index, const float* a,
+                                                        const float* s0, float* s_carry,
+                                                        float* s_lin, float* residual, int64_t B,
+                                                        int64_t D, pararnn_stream_t stream);
 
 /* ----------------------------------------------------------- decode step */
 

@@ -24,7 +24,8 @@ __all__ = [
     "pararnn_gru_adjoint",
     "pararnn_gru_adjoint_workspace_size",
     "pararnn_gru_segment_pass",
-    "pararnn_gru_segment_update",
+    "pararnn_gru_segment_fold",
+    "pararnn_gru_segment_combine",
     "pararnn_gru_sequential",
     "pararnn_gru_solve",
     "pararnn_gru_solve_async",
@@ -37,14 +38,17 @@ __all__ = [
     "pararnn_lstm_adjoint",
     "pararnn_lstm_adjoint_workspace_size",
     "pararnn_lstm_segment_pass",
-    "pararnn_lstm_segment_update",
+    "pararnn_lstm_segment_fold",
+    "pararnn_lstm_segment_combine",
     "pararnn_lstm_sequential",
     "pararnn_lstm_solve",
     "pararnn_lstm_solve_async",
     "pararnn_lstm_step",
     "pararnn_lstm_workspace_size",
     "pararnn_read_pass_times",
-    "pararnn_segment_carries",
+    "pararnn_segment_record_floats",
+    "pararnn_result_to_device",
+    "pararnn_segment_fold_workspace_size",
     "pararnn_read_result",
     "pararnn_selftest_wait_timeout",
 ]

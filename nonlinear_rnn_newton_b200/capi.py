@@ -90,9 +90,15 @@ SIGNATURES = {
                                        ctypes.c_size_t, _vp]),
     "pararnn_lstm_segment_pass": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                         ctypes.c_size_t, _vp]),
-    "pararnn_gru_segment_update": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
-    "pararnn_lstm_segment_update": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
-    "pararnn_segment_carries": (_st, [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _i64, _i64, _vp]),
+    "pararnn_result_to_device": (_st, [_vp, _vp, _vp]),
+    "pararnn_segment_record_floats": (ctypes.c_size_t, [ctypes.c_int, _i64, _i64]),
+    "pararnn_segment_fold_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _i64, _i64, _i64]),
+    "pararnn_gru_segment_fold": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
+    "pararnn_lstm_segment_fold": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
+    "pararnn_gru_segment_combine": (_st, [_vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                          _vp]),
+    "pararnn_lstm_segment_combine": (_st, [_vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                           _vp]),
     "pararnn_gru_step": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _vp]),
     "pararnn_lstm_step": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp]),
     "pararnn_linear_scan": (_st, [_vp, _st, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
@@ -516,26 +522,54 @@ def pararnn_lstm_segment_pass(u, a, s_in, s_lin, s_carry, s_out, s_end=None, wor
     _segment_pass(lib.pararnn_lstm_segment_pass, u, a, s_in, s_lin, s_carry, s_out, s_end, workspace, stream)
 
 
-def _segment_update(fn, u, a, beta, unit, carry, s_out, residual, stream):
+def pararnn_result_to_device(workspace, out, stream=None):
+    """Queue the last pass's residual and error flag into out (2 device floats)."""
+    _check(lib.pararnn_result_to_device(_ptr(workspace), _ptr(out), _stream(workspace.device, stream)), allow=(OK,))
+
+
+def pararnn_segment_record_floats(n_state, B, D):
+    return int(lib.pararnn_segment_record_floats(n_state, B, D))
+
+
+def pararnn_segment_fold_workspace_size(n_state, B, L, D):
+    return int(lib.pararnn_segment_fold_workspace_size(n_state, B, L, D))
+
+
+def _segment_fold(fn, u, a, s_in, record, workspace, stream):
     B, L, G, D = u.shape
-    st = fn(_ptr(u), _dtype_code(u), _ptr(a), _ptr(beta), _ptr(unit), _ptr(carry), _ptr(s_out), _ptr(residual),
-            B, L, D, _stream(u.device, stream))
+    st = fn(_ptr(u), _dtype_code(u), _ptr(a), _ptr(s_in), _ptr(record), B, L, D, _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(u.device, stream))
     _check(st, allow=(OK,))
 
 
-def pararnn_gru_segment_update(u, a, beta, unit, carry, h_out, residual, stream=None):
-    _segment_update(lib.pararnn_gru_segment_update, u, a, beta, unit, carry, h_out, residual, stream)
+def pararnn_gru_segment_fold(u, a, h_in, record, workspace, stream=None):
+    """The segment's record (flat, pararnn_segment_record_floats(1, B, D)) from the
+    iterate h_in [1, B, Ls, D] (None = the zero guess)."""
+    _segment_fold(lib.pararnn_gru_segment_fold, u, a, h_in, record, workspace, stream)
 
 
-def pararnn_lstm_segment_update(u, a, beta, unit, carry, s_out, residual, stream=None):
-    _segment_update(lib.pararnn_lstm_segment_update, u, a, beta, unit, carry, s_out, residual, stream)
+def pararnn_lstm_segment_fold(u, a, s_in, record, workspace, stream=None):
+    """The segment's record from the iterate s_in [2, B, Ls, D] (c, h; None = the zero guess)."""
+    _segment_fold(lib.pararnn_lstm_segment_fold, u, a, s_in, record, workspace, stream)
 
 
-def pararnn_segment_carries(ends, s0, carries, stream=None):
-    """ends [R, 1 + NS, NS, B, D], s0 [NS, B, D] or None -> carries [R, NS, B, D]."""
-    R, _, NS, B, D = ends.shape
-    st = lib.pararnn_segment_carries(_ptr(ends), _ptr(s0), _ptr(carries), R, NS, B, D, _stream(ends.device, stream))
+def _segment_combine(fn, records, index, a, s0, carry, lin, residual, stream):
+    R = records.shape[0]
+    NS, B, D = carry.shape
+    st = fn(_ptr(records), R, index, _ptr(a), _ptr(s0), _ptr(carry), _ptr(lin), _ptr(residual), B, D,
+            _stream(records.device, stream))
     _check(st, allow=(OK,))
+
+
+def pararnn_gru_segment_combine(records, index, a, h0, h_carry, h_lin, residual, stream=None):
+    """records [R, record_floats] in segment order -> h_carry, h_lin [1, B, D]
+    of segment `index` and residual (1 float) of the iterate over all segments."""
+    _segment_combine(lib.pararnn_gru_segment_combine, records, index, a, h0, h_carry, h_lin, residual, stream)
+
+
+def pararnn_lstm_segment_combine(records, index, a, s0, s_carry, s_lin, residual, stream=None):
+    """As pararnn_gru_segment_combine with states [2, B, D] (c, h)."""
+    _segment_combine(lib.pararnn_lstm_segment_combine, records, index, a, s0, s_carry, s_lin, residual, stream)
 
 
 # ------------------------------------------------------------- decode step

@@ -122,6 +122,14 @@ __device__ __forceinline__ void set_offset(Aff<2>& a, const float (&off)[2][V], 
     a.v1 = off[1][j];
 }
 
+// Set the offset part of a map from o[NS].
+__device__ __forceinline__ void set_map_offset(Aff<1>& a, const float* o) { a.v = o[0]; }
+__device__ __forceinline__ void set_map_offset(Aff<2>& a, const float* o)
+{
+    a.v0 = o[0];
+    a.v1 = o[1];
+}
+
 // Transposed map for the reverse (adjoint) recurrence mu = J^T (g + mu'):
 // matrix J^T, offset J^T g.
 __device__ __forceinline__ Aff<1> transpose_map(const Aff<1>& J, const float* g)

@@ -456,10 +456,14 @@ pararnn_status segment_pass_async(int cell, const void* u, pararnn_dtype dt, con
     TRY(check_workspace(ws, ws_bytes, solve_ws_bytes(cell, B, L, D)));
     const int NS = cell == 0 ? 1 : 2;
     const long long per = B * L * D, per0 = B * D;
-    if (s_in) {  // other CTAs overwrite what one still reads: no overlap
+    if (s_in && s_in != s_out) {
+        // in place is fine (a tile reads only its own rows, and the states
+        // entering its chunk come from the boundary rows); a shifted overlap
+        // would let one tile overwrite rows another still reads
         const uintptr_t i0 = reinterpret_cast<uintptr_t>(s_in), o0 = reinterpret_cast<uintptr_t>(s_out);
         const uintptr_t len = uintptr_t(NS * per) * 4;
-        if (i0 < o0 + len && o0 < i0 + len) return fail(PARARNN_ERR_INVALID_ARG, "s_out overlaps s_in");
+        if (i0 < o0 + len && o0 < i0 + len)
+            return fail(PARARNN_ERR_INVALID_ARG, "s_out overlaps s_in without being s_in itself");
     }
     const float* s0[2] = {s_carry, s_carry && NS == 2 ? s_carry + per0 : nullptr};
     float* st[2] = {s_out, NS == 2 ? s_out + per : nullptr};
@@ -499,39 +503,94 @@ pararnn_status segment_pass_async(int cell, const void* u, pararnn_dtype dt, con
     return PARARNN_OK;
 }
 
-pararnn_status segment_update_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* beta,
-                                    const float* unit, const float* carry, float* s_out, float* residual, long long B,
-                                    long long L, long long D, cudaStream_t stream)
+long long segment_record_floats(int cell, long long BD)
+{
+    return cell == 0 ? SegRecord<GruCell>::floats(BD) : SegRecord<LstmCell>::floats(BD);
+}
+
+// fold parts [nf][NC][B][D] of segment_fold_kernel
+size_t segment_fold_ws_bytes(int cell, long long B, long long L, long long D)
+{
+    if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
+    const long long nf = (L - 1 + kFoldSteps - 1) / kFoldSteps;
+    return align256(size_t(std::max(nf, 1ll)) * (cell == 0 ? 2 : 6) * B * D * 4);
+}
+
+template <class Cell, class UT>
+pararnn_status launch_fold(const UT* u, const float* a, const float* s_in, float* rec, float* part, long long B,
+                           long long L, long long D, cudaStream_t stream)
+{
+    using R = SegRecord<Cell>;
+    const long long BD = B * D;
+    unsigned* res = reinterpret_cast<unsigned*>(rec + R::F * BD);
+    CUDA_TRY(cudaMemsetAsync(res, 0, 16, stream));
+    const int nf = int((L - 1 + kFoldSteps - 1) / kFoldSteps);
+    if (nf > 0) {
+        const long long threads = B * (D / 4);
+        const dim3 grid(unsigned((threads + 127) / 128), unsigned(nf)), block(128);
+        segment_fold_kernel<Cell, UT><<<grid, block, 0, stream>>>(u, a, s_in, part, res, B, L, D);
+        CUDA_TRY(cudaGetLastError());
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+    segment_record_kernel<Cell, UT><<<unsigned((BD + 255) / 256), 256, 0, stream>>>(u, s_in, part, nf, rec, B, L, D);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
+// A segment's record for the iteration from H^k = s_in [NS][B][Ls][D] (NULL:
+// the zero guess): see SegRecord in segment.cuh.
+pararnn_status segment_fold_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* s_in,
+                                  float* rec, long long B, long long L, long long D, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream)
 {
     t_err[0] = '\0';
     TRY(check_dtype(dt));
     TRY(check_ptr(u, "u", true));
     TRY(check_ptr(a, "a", true));
-    TRY(check_ptr(beta, "beta", true));
-    TRY(check_ptr(unit, "unit", true));
-    TRY(check_ptr(carry, "carry", true));
-    TRY(check_ptr(s_out, "s_out", true));
-    if (!residual) return fail(PARARNN_ERR_INVALID_ARG, "residual is NULL");
+    TRY(check_ptr(s_in, "s_in", false));
+    TRY(check_ptr(rec, "record", true));
     Shape s;
     TRY(make_shape(B, L, D, 1, &s));
-    const long long n = B * L * D;
-    const dim3 grid(unsigned((n + 255) / 256)), block(256);
-    unsigned* res = reinterpret_cast<unsigned*>(residual);
+    TRY(check_workspace(ws, ws_bytes, segment_fold_ws_bytes(cell, B, L, D)));
+    float* part = static_cast<float*>(ws);
     if (cell == 0) {
         if (dt == PARARNN_BF16)
-            segment_update_kernel<GruCell, uint16_t><<<grid, block, 0, stream>>>(
-                static_cast<const uint16_t*>(u), a, beta, unit, carry, s_out, res, B, L, D);
-        else
-            segment_update_kernel<GruCell, float><<<grid, block, 0, stream>>>(static_cast<const float*>(u), a, beta,
-                                                                              unit, carry, s_out, res, B, L, D);
-    } else {
-        if (dt == PARARNN_BF16)
-            segment_update_kernel<LstmCell, uint16_t><<<grid, block, 0, stream>>>(
-                static_cast<const uint16_t*>(u), a, beta, unit, carry, s_out, res, B, L, D);
-        else
-            segment_update_kernel<LstmCell, float><<<grid, block, 0, stream>>>(static_cast<const float*>(u), a, beta,
-                                                                               unit, carry, s_out, res, B, L, D);
+            return launch_fold<GruCell, uint16_t>(static_cast<const uint16_t*>(u), a, s_in, rec, part, B, L, D, stream);
+        return launch_fold<GruCell, float>(static_cast<const float*>(u), a, s_in, rec, part, B, L, D, stream);
     }
+    if (dt == PARARNN_BF16)
+        return launch_fold<LstmCell, uint16_t>(static_cast<const uint16_t*>(u), a, s_in, rec, part, B, L, D, stream);
+    return launch_fold<LstmCell, float>(static_cast<const float*>(u), a, s_in, rec, part, B, L, D, stream);
+}
+
+// Every segment's record (R of them, in segment order) -> the state entering
+// segment `index` and the state its first step is linearised at, and the
+// residual of the iterate over all segments.
+pararnn_status segment_combine_async(int cell, const float* recs, int n_seg, int index, const float* a,
+                                     const float* s0, float* carry, float* lin, float* residual, long long B,
+                                     long long D, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_ptr(recs, "records", true));
+    TRY(check_ptr(a, "a", true));
+    TRY(check_ptr(s0, "s0", false));
+    TRY(check_ptr(carry, "carry", true));
+    TRY(check_ptr(lin, "lin", true));
+    if (!residual) return fail(PARARNN_ERR_INVALID_ARG, "residual is NULL");
+    if (n_seg < 1) return fail(PARARNN_ERR_INVALID_ARG, "n_segments must be >= 1 (got %d)", n_seg);
+    if (index < 0 || index >= n_seg)
+        return fail(PARARNN_ERR_INVALID_ARG, "index %d is not a segment of %d", index, n_seg);
+    if (B < 1 || D < 1 || D % 8 != 0) return fail(B < 1 || D < 1 ? PARARNN_ERR_INVALID_ARG : PARARNN_ERR_UNSUPPORTED,
+                                                  "B, D must be >= 1 and D a multiple of 8");
+    const long long BD = B * D;
+    unsigned* res = reinterpret_cast<unsigned*>(residual);
+    CUDA_TRY(cudaMemsetAsync(res, 0, 4, stream));
+    const dim3 grid(unsigned((BD + 255) / 256)), block(256);
+    if (cell == 0)
+        segment_combine_kernel<GruCell><<<grid, block, 0, stream>>>(recs, n_seg, index, s0, a, carry, lin, res, B, D);
+    else
+        segment_combine_kernel<LstmCell><<<grid, block, 0, stream>>>(recs, n_seg, index, s0, a, carry, lin, res, B, D);
     CUDA_TRY(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return PARARNN_OK;
@@ -932,6 +991,18 @@ pararnn_status pararnn_read_result(const void* workspace, pararnn_stream_t strea
     return pararnn_status(r.status);
 }
 
+pararnn_status pararnn_result_to_device(const void* workspace, float* out, pararnn_stream_t stream)
+{
+    t_err[0] = '\0';
+    if (!workspace) return fail(PARARNN_ERR_WORKSPACE, "workspace is NULL");
+    if (!out) return fail(PARARNN_ERR_INVALID_ARG, "out is NULL");
+    result_outcome_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const WsHeader*>(workspace), out);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
 // ------------------------------------------------------------- adjoints
 
 size_t pararnn_gru_adjoint_workspace_size(int64_t B, int64_t L, int64_t D) { return adjoint_ws_bytes(0, B, L, D); }
@@ -1070,42 +1141,48 @@ pararnn_status pararnn_lstm_segment_pass(const void* u, pararnn_dtype u_dtype, c
                               workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
-pararnn_status pararnn_gru_segment_update(const void* u, pararnn_dtype u_dtype, const float* a, const float* beta,
-                                          const float* unit, const float* carry, float* h_out, float* residual,
-                                          int64_t B, int64_t L, int64_t D, pararnn_stream_t stream)
+size_t pararnn_segment_record_floats(int n_state, int64_t B, int64_t D)
 {
-    return segment_update_async(0, u, u_dtype, a, beta, unit, carry, h_out, residual, B, L, D,
-                                reinterpret_cast<cudaStream_t>(stream));
+    if ((n_state != 1 && n_state != 2) || B < 1 || D < 1) return 0;
+    return size_t(segment_record_floats(n_state - 1, (long long)B * D));
 }
 
-pararnn_status pararnn_lstm_segment_update(const void* u, pararnn_dtype u_dtype, const float* a, const float* beta,
-                                           const float* unit, const float* carry, float* s_out, float* residual,
-                                           int64_t B, int64_t L, int64_t D, pararnn_stream_t stream)
+size_t pararnn_segment_fold_workspace_size(int n_state, int64_t B, int64_t L, int64_t D)
 {
-    return segment_update_async(1, u, u_dtype, a, beta, unit, carry, s_out, residual, B, L, D,
-                                reinterpret_cast<cudaStream_t>(stream));
+    if (n_state != 1 && n_state != 2) return 0;
+    return segment_fold_ws_bytes(n_state - 1, B, L, D);
 }
 
-pararnn_status pararnn_segment_carries(const float* ends, const float* s0, float* carries, int n_segments,
-                                       int n_state, int64_t B, int64_t D, pararnn_stream_t stream)
+pararnn_status pararnn_gru_segment_fold(const void* u, pararnn_dtype u_dtype, const float* a, const float* h_in,
+                                        float* record, int64_t B, int64_t L, int64_t D, void* workspace,
+                                        size_t workspace_bytes, pararnn_stream_t stream)
 {
-    t_err[0] = '\0';
-    TRY(check_ptr(ends, "ends", true));
-    TRY(check_ptr(s0, "s0", false));
-    TRY(check_ptr(carries, "carries", true));
-    if (n_segments < 1) return fail(PARARNN_ERR_INVALID_ARG, "n_segments must be >= 1 (got %d)", n_segments);
-    if (n_state != 1 && n_state != 2) return fail(PARARNN_ERR_INVALID_ARG, "n_state must be 1 or 2 (got %d)", n_state);
-    if (B < 1 || D < 1) return fail(PARARNN_ERR_INVALID_ARG, "B, D must be >= 1");
-    const long long BD = (long long)B * D;
-    const dim3 grid(unsigned((BD + 255) / 256)), block(256);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (n_state == 1)
-        segment_carries_kernel<1><<<grid, block, 0, st>>>(ends, s0, carries, n_segments, BD);
-    else
-        segment_carries_kernel<2><<<grid, block, 0, st>>>(ends, s0, carries, n_segments, BD);
-    CUDA_TRY(cudaGetLastError());
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return PARARNN_OK;
+    return segment_fold_async(0, u, u_dtype, a, h_in, record, B, L, D, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_lstm_segment_fold(const void* u, pararnn_dtype u_dtype, const float* a, const float* s_in,
+                                         float* record, int64_t B, int64_t L, int64_t D, void* workspace,
+                                         size_t workspace_bytes, pararnn_stream_t stream)
+{
+    return segment_fold_async(1, u, u_dtype, a, s_in, record, B, L, D, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_gru_segment_combine(const float* records, int n_segments, int index, const float* a,
+                                           const float* h0, float* h_carry, float* h_lin, float* residual, int64_t B,
+                                           int64_t D, pararnn_stream_t stream)
+{
+    return segment_combine_async(0, records, n_segments, index, a, h0, h_carry, h_lin, residual, B, D,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_lstm_segment_combine(const float* records, int n_segments, int index, const float* a,
+                                            const float* s0, float* s_carry, float* s_lin, float* residual,
+                                            int64_t B, int64_t D, pararnn_stream_t stream)
+{
+    return segment_combine_async(1, records, n_segments, index, a, s0, s_carry, s_lin, residual, B, D,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t pararnn_linear_scan_workspace_size(int64_t B, int64_t L, int64_t D) { return linear_scan_ws_bytes(B, L, D); }

@@ -3,13 +3,14 @@
 //
 // Page: "ParaRNN: Apple destrava treino paralelo de RNNs não-lineares e escala
 // pra 7B parâmetros" -- "A sacada: método de Newton": each iteration solves a
-// linear recurrence s^{k+1}_l = J_l s^{k+1}_{l-1} + o_l.  Over a segment that
-// starts after step l0 - 1 its solution is affine in the state entering the
-// segment, c = s^{k+1}_{l0-1}:  s^{k+1}_l = beta_l + A_l c.  One pass with
-// c = 0 gives beta, one pass with c = e_j per state component gives
-// beta + A e_j; the maps of the segments' last steps, gathered from every
-// GPU and composed in order, give each segment its c (a scan over segments),
-// and a fix-up writes s^{k+1} = beta + A c and the residual of the result.
+// linear recurrence s^{k+1}_l = J_l s^{k+1}_{l-1} + o_l whose step maps
+// depend only on the iterate H^k.  Over a segment their composition is one
+// affine map of the state entering the segment.  Per iteration each GPU folds
+// its segment's step maps (segment_fold_kernel, segment_record_kernel), the
+// segments' records are gathered from every GPU (the one data exchange), and
+// every GPU composes them in order into the state entering its own segment
+// (segment_combine_kernel); one fused pass in segment mode then writes the
+// segment's next iterate and its residual.
 #pragma once
 
 #include "cells.cuh"
@@ -43,100 +44,231 @@ __global__ void __launch_bounds__(256) bnd_gather_kernel(const float* __restrict
 __device__ __forceinline__ float gate_value(const uint16_t* p) { return __uint_as_float(uint32_t(*p) << 16); }
 __device__ __forceinline__ float gate_value(const float* p) { return *p; }
 
-// s = beta + sum_j (unit_j - beta) c_j over the segment, and max |F| of the
-// result, F_l = s_l - f(s_{l-1}, u_l) with s_{-1} = c.
-//   beta [NS][B][L][D], unit [NS (j)][NS][B][L][D] (the pass with c = e_j),
-//   carry [NS][B][D], out [NS][B][L][D], res: max |F| as float bits
-//   (non-negative floats order like their bits; NaN kept).
-// One thread per (b, l, d).
-template <class Cell, class UT>
-__global__ void __launch_bounds__(256) segment_update_kernel(const UT* __restrict__ u, const float* __restrict__ a,
-                                                             const float* __restrict__ beta,
-                                                             const float* __restrict__ unit,
-                                                             const float* __restrict__ carry, float* __restrict__ out,
-                                                             unsigned* res, long long B, long long L, long long D)
+__device__ __forceinline__ float max_nan(float a, float b) { return (b > a || b != b) ? b : a; }
+
+// Block-wide maximum (NaN kept) folded into *res as float bits
+// (non-negative floats order like their bits).
+__device__ __forceinline__ void block_max_into(float v, unsigned* res)
 {
-    constexpr int G = Cell::G, NS = Cell::NS;
-    const long long per = B * L * D;
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    float emax = 0.f;
-    if (i < per) {
-        const long long d = i % D, bl = i / D, b = bl / L, l = bl - b * L;
-        float c[NS];
 #pragma unroll
-        for (int q = 0; q < NS; ++q) c[q] = carry[(q * B + b) * D + d];
-        auto fix = [&](long long idx, int q) {
-            const float be = beta[q * per + idx];
-            float v = be;
-#pragma unroll
-            for (int j = 0; j < NS; ++j) v = fmaf(unit[(j * NS + q) * per + idx] - be, c[j], v);
-            return v;
-        };
-        float cur[NS], prv[NS], uu[G], aa[G], f[NS];
-#pragma unroll
-        for (int q = 0; q < NS; ++q) {
-            cur[q] = fix(i, q);
-            prv[q] = l > 0 ? fix(i - D, q) : c[q];
-            out[q * per + i] = cur[q];
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            uu[g] = gate_value(u + (bl * G + g) * D + d);
-            aa[g] = a[g * D + d];
-        }
-        Cell::value(prv, uu, aa, f);
-#pragma unroll
-        for (int q = 0; q < NS; ++q) {
-            const float e = fabsf(cur[q] - f[q]);
-            emax = (e > emax || e != e) ? e : emax;
-        }
-    }
-    // block maximum, NaN kept
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const float o = __shfl_xor_sync(0xffffffffu, emax, off);
-        emax = (o > emax || o != o) ? o : emax;
-    }
-    __shared__ float wmax[8];
-    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = emax;
+    for (int off = 16; off > 0; off >>= 1) v = max_nan(v, __shfl_xor_sync(0xffffffffu, v, off));
+    __shared__ float wmax[32];
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = v;
     __syncthreads();
     if (threadIdx.x == 0) {
         float m = 0.f;
-        for (int w = 0; w < int(blockDim.x >> 5); ++w) m = (wmax[w] > m || wmax[w] != wmax[w]) ? wmax[w] : m;
+        for (int w = 0; w < int((blockDim.x + 31) >> 5); ++w) m = max_nan(m, wmax[w]);
         atomicMax(res, __float_as_uint(m) & 0x7fffffffu);
     }
 }
 
-// The state entering every segment, from the segments' last-step values:
-//   ends [R][1 + NS][NS][B][D]: per segment, its last step's state in the
-//   pass with c = 0 (beta) and in the passes with c = e_j;
-//   s0 [NS][B][D] (NULL = zeros) enters segment 0;
-//   carries [R][NS][B][D]: c_0 = s0, c_{r+1} = beta_r + sum_j (unit_rj - beta_r) c_r[j].
-template <int NS>
-__global__ void __launch_bounds__(256) segment_carries_kernel(const float* __restrict__ ends,
-                                                              const float* __restrict__ s0,
-                                                              float* __restrict__ carries, int R, long long BD)
+// Record a segment contributes to an iteration of the split solve, per
+// channel, fields [F][B][D] with F = NC + 2 NS + G, then one float:
+//   fold  [NC]: the composition of the step maps s -> J_l s + o_l of steps
+//               1..Ls-1 of the segment (identity if Ls = 1), linearised at
+//               the iterate H^k;
+//   last  [NS]: H^k at the segment's last step (the next segment's first
+//               step is linearised there);
+//   first [NS]: H^k at the segment's first step;
+//   gates [G]:  the first step's gate pre-activations (fp32);
+//   then max |F_l(H^k)| over steps 1..Ls-1 (float, NaN kept).
+template <class Cell>
+struct SegRecord {
+    static constexpr int NC = Cell::Map::kFloats, NS = Cell::NS, G = Cell::G;
+    static constexpr int F = NC + 2 * NS + G;
+    static constexpr int fold = 0, last = NC, first = NC + NS, gates = NC + 2 * NS;
+    static __host__ __device__ long long floats(long long BD) { return F * BD + 4; }
+};
+
+// Steps folded per thread in segment_fold_kernel.
+constexpr int kFoldSteps = 128;
+
+// Fold of steps [1 + f*kFoldSteps, 1 + (f+1)*kFoldSteps) of a segment (f =
+// blockIdx.y) for 4 channels a thread: the step maps at H^k (s_in, NULL = the
+// zero guess) composed in order into part [nf][NC][B][D], and max |F| of the
+// steps into *res.  Page: "A sacada: método de Newton" (the Newton step is the
+// linear recurrence s^{k+1}_l = J_l s^{k+1}_{l-1} + o_l, o_l = f_l - J_l s^k_{l-1}).
+template <class Cell, class UT>
+__global__ void __launch_bounds__(128) segment_fold_kernel(const UT* __restrict__ u, const float* __restrict__ a,
+                                                           const float* __restrict__ s_in, float* __restrict__ part,
+                                                           unsigned* res, long long B, long long Ls, long long D)
 {
+    using Map = typename Cell::Map;
+    constexpr int G = Cell::G, NS = Cell::NS, NC = Map::kFloats;
+    const long long D4 = D >> 2, BD = B * D, per = B * Ls * D;
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= BD) return;
-    float c[NS];
+    float rmax = 0.f;
+    if (i < B * D4) {
+        const long long b = i / D4, d = (i - b * D4) << 2;
+        const long long l0 = 1 + (long long)blockIdx.y * kFoldSteps;
+        const long long l1 = l0 + kFoldSteps < Ls ? l0 + kFoldSteps : Ls;
+        float av[G][kV];
 #pragma unroll
-    for (int q = 0; q < NS; ++q) c[q] = s0 ? s0[q * BD + i] : 0.f;
-    for (int r = 0; r < R; ++r) {
-        float nc[NS];
+        for (int g = 0; g < G; ++g) {
+            const F4 x = load4(a + g * D + d);
+#pragma unroll
+            for (int j = 0; j < kV; ++j) av[g][j] = x.v[j];
+        }
+        float prev[NS][kV];
 #pragma unroll
         for (int q = 0; q < NS; ++q) {
-            carries[((long long)r * NS + q) * BD + i] = c[q];
-            const float be = ends[((long long)r * (1 + NS) * NS + q) * BD + i];
-            float v = be;
+            F4 x{{0.f, 0.f, 0.f, 0.f}};
+            if (s_in) x = load4(s_in + q * per + (b * Ls + l0 - 1) * D + d);
 #pragma unroll
-            for (int j = 0; j < NS; ++j)
-                v = fmaf(ends[(((long long)r * (1 + NS) + 1 + j) * NS + q) * BD + i] - be, c[j], v);
-            nc[q] = v;
+            for (int j = 0; j < kV; ++j) prev[q][j] = x.v[j];
+        }
+        Map acc[kV];
+#pragma unroll
+        for (int j = 0; j < kV; ++j) acc[j] = Map::identity();
+        // unrolled so that the loads of several steps are in flight together
+#pragma unroll 4
+        for (long long l = l0; l < l1; ++l) {
+            F4 ug[G], cur[NS];
+#pragma unroll
+            for (int g = 0; g < G; ++g) ug[g] = load4(u + ((b * Ls + l) * G + g) * D + d);
+#pragma unroll
+            for (int q = 0; q < NS; ++q) {
+                cur[q] = F4{{0.f, 0.f, 0.f, 0.f}};
+                if (s_in) cur[q] = load4(s_in + q * per + (b * Ls + l) * D + d);
+            }
+#pragma unroll
+            for (int j = 0; j < kV; ++j) {
+                float sp[NS], uu[G], aa[G], f[NS], js[NS];
+#pragma unroll
+                for (int q = 0; q < NS; ++q) sp[q] = prev[q][j];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    uu[g] = ug[g].v[j];
+                    aa[g] = av[g][j];
+                }
+                Map m;
+                Cell::eval(sp, uu, aa, f, m);
+                apply_matrix(m, sp, js);
+                float o[NS];
+#pragma unroll
+                for (int q = 0; q < NS; ++q) {
+                    o[q] = f[q] - js[q];
+                    rmax = max_nan(rmax, fabsf(cur[q].v[j] - f[q]));
+                    prev[q][j] = cur[q].v[j];
+                }
+                set_map_offset(m, o);
+                acc[j] = compose(m, acc[j]);
+            }
         }
 #pragma unroll
-        for (int q = 0; q < NS; ++q) c[q] = nc[q];
+        for (int c = 0; c < NC; ++c) {
+            float v[kV];
+#pragma unroll
+            for (int j = 0; j < kV; ++j) v[j] = acc[j].get(c);
+            store4(part + ((long long)blockIdx.y * NC + c) * BD + b * D + d, v);
+        }
     }
+    block_max_into(rmax, res);
+}
+
+// The segment's record (SegRecord) from the fold parts: the parts composed in
+// order, H^k at the first and last steps, the first step's gates.  One
+// thread per channel.
+template <class Cell, class UT>
+__global__ void __launch_bounds__(256) segment_record_kernel(const UT* __restrict__ u, const float* __restrict__ s_in,
+                                                             const float* __restrict__ part, int nf,
+                                                             float* __restrict__ rec, long long B, long long Ls,
+                                                             long long D)
+{
+    using Map = typename Cell::Map;
+    using R = SegRecord<Cell>;
+    constexpr int G = Cell::G, NS = Cell::NS, NC = Map::kFloats;
+    const long long BD = B * D, per = B * Ls * D;
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= BD) return;
+    const long long b = i / D, d = i - b * D;
+    Map acc = Map::identity();
+    for (int f = 0; f < nf; ++f) {
+        Map m;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) m.set(c, part[((long long)f * NC + c) * BD + i]);
+        acc = compose(m, acc);
+    }
+#pragma unroll
+    for (int c = 0; c < NC; ++c) rec[(R::fold + c) * BD + i] = acc.get(c);
+#pragma unroll
+    for (int q = 0; q < NS; ++q) {
+        rec[(R::last + q) * BD + i] = s_in ? s_in[q * per + (b * Ls + Ls - 1) * D + d] : 0.f;
+        rec[(R::first + q) * BD + i] = s_in ? s_in[q * per + (b * Ls) * D + d] : 0.f;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) rec[(R::gates + g) * BD + i] = gate_value(u + (b * Ls * G + g) * D + d);
+}
+
+// Every segment's record gathered, in segment order (R records of
+// SegRecord::floats(B*D) floats each) -> for segment `me`: the state entering
+// it at iterate k+1 (carry) and the iterate's state before it (lin, where its
+// first step is linearised), both [NS][B][D]; and max |F(H^k)| over all
+// segments into *res.  Page: "A sacada: método de Newton" -- the Newton
+// linear recurrence composed segment by segment: segment j maps the state c
+// entering it to fold_j(J (c - lin_j) + f(lin_j, u_j1)), with J = df/ds at
+// lin_j, the previous segment's last iterate state (s0 for segment 0).
+template <class Cell>
+__global__ void __launch_bounds__(256) segment_combine_kernel(const float* __restrict__ recs, int n_seg, int me,
+                                                              const float* __restrict__ s0, const float* __restrict__ a,
+                                                              float* __restrict__ carry, float* __restrict__ lin_out,
+                                                              unsigned* res, long long B, long long D)
+{
+    using Map = typename Cell::Map;
+    using R = SegRecord<Cell>;
+    constexpr int G = Cell::G, NS = Cell::NS, NC = Map::kFloats;
+    const long long BD = B * D, RF = R::floats(BD);
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    float rmax = 0.f;
+    if (i < BD) {
+        const long long d = i % D;
+        float aa[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) aa[g] = a[g * D + d];
+        float c[NS], lin[NS];
+#pragma unroll
+        for (int q = 0; q < NS; ++q) c[q] = lin[q] = s0 ? s0[q * BD + i] : 0.f;
+        for (int j = 0; j < n_seg; ++j) {
+            const float* rj = recs + j * RF;
+            float uu[G], f[NS], x[NS], dl[NS], jx[NS];
+#pragma unroll
+            for (int g = 0; g < G; ++g) uu[g] = rj[(R::gates + g) * BD + i];
+            Map m;
+            Cell::eval(lin, uu, aa, f, m);
+#pragma unroll
+            for (int q = 0; q < NS; ++q) {
+                rmax = max_nan(rmax, fabsf(rj[(R::first + q) * BD + i] - f[q]));
+                if (j == me) {
+                    carry[q * BD + i] = c[q];
+                    lin_out[q * BD + i] = lin[q];
+                }
+                dl[q] = c[q] - lin[q];
+            }
+            apply_matrix(m, dl, jx);
+#pragma unroll
+            for (int q = 0; q < NS; ++q) x[q] = jx[q] + f[q];
+            Map fold;
+#pragma unroll
+            for (int k = 0; k < NC; ++k) fold.set(k, rj[(R::fold + k) * BD + i]);
+            apply(fold, x, c);
+#pragma unroll
+            for (int q = 0; q < NS; ++q) lin[q] = rj[(R::last + q) * BD + i];
+        }
+    }
+    if (i == 0) {  // the segments' own maxima over their steps 1..Ls-1
+        for (int j = 0; j < n_seg; ++j) rmax = max_nan(rmax, recs[j * RF + R::F * BD]);
+    }
+    block_max_into(rmax, res);
+}
+
+// The outcome of the last fused pass on a workspace as device floats:
+// out[0] = the residual it published, out[1] = 1 if a device-side error was
+// raised, else 0 (so that a host loop can reduce both across GPUs without
+// reading the header first).
+__global__ void result_outcome_kernel(const WsHeader* hdr, float* out)
+{
+    out[0] = hdr->result.residual;
+    out[1] = hdr->error != 0 ? 1.f : 0.f;
 }
 
 }  // namespace pararnn

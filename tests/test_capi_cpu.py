@@ -117,13 +117,28 @@ def test_segment_checks(capi):
     assert "overlaps" in capi.last_error()
     assert lib.pararnn_lstm_segment_pass(16, 1, 16, None, None, None, None, None, 1, 8, 16, 256, 1 << 20,
                                          None) == E.ERR_INVALID_ARG
-    upd = lambda res=4096, D=16: lib.pararnn_gru_segment_update(16, 1, 16, 16, 16, 16, 16, res, 1, 8, D, None)
-    assert upd(res=None) == E.ERR_INVALID_ARG
-    assert upd(D=12) == E.ERR_UNSUPPORTED
-    car = lambda R=2, NS=1, B=1, D=16: lib.pararnn_segment_carries(16, None, 16, R, NS, B, D, None)
-    assert car(R=0) == E.ERR_INVALID_ARG
-    assert car(NS=3) == E.ERR_INVALID_ARG
-    assert car(B=0) == E.ERR_INVALID_ARG
+    fold = lambda u=16, rec=4096, D=16, ws=256, wsb=1 << 20: lib.pararnn_gru_segment_fold(
+        u, 1, 16, None, rec, 1, 8, D, ws, wsb, None)
+    assert fold(u=None) == E.ERR_INVALID_ARG
+    assert fold(rec=None) == E.ERR_INVALID_ARG
+    assert fold(D=12) == E.ERR_UNSUPPORTED
+    assert fold(ws=None) == E.ERR_WORKSPACE
+    assert fold(wsb=16) == E.ERR_WORKSPACE
+    comb = lambda R=2, i=0, res=4096, B=1, D=16: lib.pararnn_gru_segment_combine(16, R, i, 16, None, 16, 16, res,
+                                                                                  B, D, None)
+    assert comb(R=0) == E.ERR_INVALID_ARG
+    assert comb(i=2) == E.ERR_INVALID_ARG
+    assert comb(res=None) == E.ERR_INVALID_ARG
+    assert comb(B=0) == E.ERR_INVALID_ARG
+    assert comb(D=12) == E.ERR_UNSUPPORTED
+    # record: F = NC + 2 NS + G fields of B*D floats, then 4 floats
+    assert lib.pararnn_segment_record_floats(1, 2, 16) == (2 + 2 + 3) * 32 + 4
+    assert lib.pararnn_segment_record_floats(2, 2, 16) == (6 + 4 + 4) * 32 + 4
+    assert lib.pararnn_segment_record_floats(3, 2, 16) == 0
+    # partial folds of 128 steps: steps 2..L of the segment
+    assert lib.pararnn_segment_fold_workspace_size(1, 1, 129, 16) == 256
+    assert lib.pararnn_segment_fold_workspace_size(2, 4, 257, 64) == 2 * 6 * 4 * 64 * 4
+    assert lib.pararnn_segment_fold_workspace_size(2, 4, 258, 64) == 3 * 6 * 4 * 64 * 4
 
 
 def test_decode_step_checks(capi):

@@ -75,5 +75,22 @@ def test_segment_stopping_rules(cuda):
     Hs = torch.cat([sg.H for sg in segs], dim=2)[0]
     assert it == 1 and st == 1 and H.max_abs(Hs.cpu(), h1) <= 1e-4
     from nonlinear_rnn_newton_b200 import capi
-    with pytest.raises(capi.PararnnError):  # output overlapping the iterate it reads
-        P().pararnn_gru_segment_pass(segs[0].u, xd.a, segs[0].H, None, None, segs[0].H, None, segs[0].ws)
+    with pytest.raises(capi.PararnnError):  # output overlapping the iterate it reads, shifted by one row
+        P().pararnn_gru_segment_pass(segs[0].u, xd.a, segs[0].H, None, None, segs[0].H.view(-1)[64:], None,
+                                     segs[0].ws)
+
+
+def test_segment_memory_is_the_iterate_plus_small_buffers(cuda):
+    """A segment holds its iterate (updated in place), B*D-sized buffers, the
+    fold's partial maps (one per 128 steps) and the fused pass's workspace:
+    nothing else of the iterate's size."""
+    B, Ls, D = 2, 1024, 256
+    u = torch.zeros((B, Ls, 3, D), dtype=torch.bfloat16, device=cuda)
+    a = torch.zeros((3, D), device=cuda)
+    sg = SH.Segment("gru", u, a, 0)
+    state = sg.H.numel() * 4
+    extra = sg.rec.numel() * 4 + sg.carry.numel() * 4 + sg.lin.numel() * 4 + sg.res.numel() * 4
+    assert sg.H.shape == (1, B, Ls, D) and extra <= 16 * B * D * 4
+    assert sg.ws.numel() == max(P().pararnn_gru_workspace_size(B, Ls, D),
+                                P().pararnn_segment_fold_workspace_size(1, B, Ls, D))
+    assert P().pararnn_segment_fold_workspace_size(1, B, Ls, D) <= state // 32

@@ -1,12 +1,13 @@
 """The host logic of the sequence-split solve (nonlinear_rnn_newton_b200.sharded)
 on CPU ranks (gloo, world size 2 and 3): every rank holds one segment, the
-segments' ends are all-gathered in segment order, the residual maximum is
+segments' records are all-gathered in segment order, the residual maximum is
 all-reduced, and the stopping decision is common.  The per-segment
-computations are a float64 stand-in written here from the method (one Newton
-pass over a segment from a linearisation point and a carry; the affine
-fix-up; the composition of the segments' maps), so the test checks the
-orchestration and the algebra, not the kernels (which the GPU tests check).
-Expected: the oracle's sequential states and its Newton iteration count."""
+computations are a float64 stand-in written here from the method (the fold
+of a segment's step maps at the iterate; their composition segment by segment
+into the state entering each one; one Newton pass over a segment from its
+linearisation point and carry), so the test checks the orchestration and the
+algebra, not the kernels (which the GPU tests check).  Expected: the oracle's
+sequential states and its Newton iteration count."""
 import os
 import socket
 
@@ -20,66 +21,89 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 class Float64Segment:
-    """The interface of sharded.Segment, computed in float64 on the CPU."""
+    """The interface of sharded.Segment, computed in float64 on the CPU.
+    Record (flat): fold matrix M [NS][NS][B][D], fold offset v [NS][B][D],
+    last and first iterate states [NS][B][D] each, first-step gates
+    [G][B][D], then the residual over steps 2..Ls."""
 
     def __init__(self, cell, u, a, index):
         self.cell, self.index, self.stream = cell, index, None
         self.step, self.jac = cell.step, cell.jac
-        self.NS = cell.NS
-        self.u = u                                   # [B, Ls, G, D] float64
+        self.NS, self.G = cell.NS, cell.G
         self.a = a.numpy()
         self.ug = np.transpose(u.numpy(), (1, 2, 0, 3))  # [Ls, G, B, D]
         B, Ls, G, D = u.shape
+        self.B, self.Ls, self.D = B, Ls, D
         self.H = torch.zeros((self.NS, B, Ls, D), dtype=torch.float64)
-        self.P = np.zeros((1 + self.NS, self.NS, B, Ls, D))
-        self.ends = torch.zeros((1 + self.NS, self.NS, B, D), dtype=torch.float64)
+        self.carry = np.zeros((self.NS, B, D))
         self.lin = np.zeros((self.NS, B, D))
-        self.res = torch.zeros(1, dtype=torch.float64)
+        self.res = 0.0
 
-    def _residual(self, Hn, prev0):
-        prev, r = prev0, 0.0
-        for l in range(Hn.shape[2]):
-            # NaN kept, like the kernels' max.NaN (Python's max would drop it)
-            r = float(np.maximum(r, np.max(np.abs(Hn[:, :, l] - self.step(prev, self.ug[l], self.a)))))
-            prev = Hn[:, :, l]
-        return r
+    def _map(self, prev, l):
+        J = self.jac(prev, self.ug[l], self.a)                 # [NS][NS][B][D]
+        f = self.step(prev, self.ug[l], self.a)
+        return J, f - np.einsum("qrbd,rbd->qbd", J, prev)
 
     def start(self, s0):
         self.H.zero_()
-        self.lin = s0.numpy().copy() if (self.index == 0 and s0 is not None) else np.zeros_like(self.lin)
-        self.res[0] = self._residual(self.H.numpy(), self.lin)
 
-    def passes(self, k):
+    def fold(self, k):
         Hk = self.H.numpy()
-        for j in range(1 + self.NS):
-            c = np.zeros_like(self.lin)
-            if j > 0:
-                c[j - 1] = 1.0
-            prev_k, s = self.lin, c
-            for l in range(Hk.shape[2]):
-                J = self.jac(prev_k, self.ug[l], self.a)
-                f = self.step(prev_k, self.ug[l], self.a)
-                o = f - np.einsum("qrbd,rbd->qbd", J, prev_k)
-                s = np.einsum("qrbd,rbd->qbd", J, s) + o
-                self.P[j, :, :, l] = s
-                prev_k = Hk[:, :, l]
-            self.ends[j] = torch.from_numpy(self.P[j, :, :, -1].copy())
+        NS, B, D = self.NS, self.B, self.D
+        M = np.broadcast_to(np.eye(NS)[:, :, None, None], (NS, NS, B, D)).copy()
+        v = np.zeros((NS, B, D))
+        r = 0.0
+        for l in range(1, self.Ls):
+            J, o = self._map(Hk[:, :, l - 1], l)
+            M = np.einsum("qrbd,rsbd->qsbd", J, M)
+            v = np.einsum("qrbd,rbd->qbd", J, v) + o
+            f = self.step(Hk[:, :, l - 1], self.ug[l], self.a)
+            r = float(np.maximum(r, np.max(np.abs(Hk[:, :, l] - f))))
+        parts = [M.ravel(), v.ravel(), Hk[:, :, -1].ravel(), Hk[:, :, 0].ravel(), self.ug[0].ravel(), [r, 0, 0, 0]]
+        self.rec = torch.from_numpy(np.concatenate(parts))
 
-    def carries(self, ends, s0):
-        e = ends.numpy()
-        c = s0.numpy().copy() if s0 is not None else np.zeros(e.shape[2:])
-        out = np.empty((e.shape[0],) + c.shape)
-        for r in range(e.shape[0]):
-            out[r] = c
-            c = e[r, 0] + sum((e[r, 1 + j] - e[r, 0]) * c[j] for j in range(self.NS))
-        return torch.from_numpy(out)
+    def combine(self, recs, s0):
+        NS, G, B, D = self.NS, self.G, self.B, self.D
+        c = s0.numpy().copy() if s0 is not None else np.zeros((NS, B, D))
+        lin = c.copy()
+        r = 0.0
+        for j, rec in enumerate(recs.numpy()):
+            o = 0
+            M = rec[o:o + NS * NS * B * D].reshape(NS, NS, B, D); o += NS * NS * B * D
+            v = rec[o:o + NS * B * D].reshape(NS, B, D); o += NS * B * D
+            last = rec[o:o + NS * B * D].reshape(NS, B, D); o += NS * B * D
+            first = rec[o:o + NS * B * D].reshape(NS, B, D); o += NS * B * D
+            u1 = rec[o:o + G * B * D].reshape(G, B, D); o += G * B * D
+            r = float(np.maximum(r, rec[o]))
+            J = self.jac(lin, u1, self.a)
+            f = self.step(lin, u1, self.a)
+            r = float(np.maximum(r, np.max(np.abs(first - f))))
+            if j == self.index:
+                self.carry, self.lin = c.copy(), lin.copy()
+            x = np.einsum("qrbd,rbd->qbd", J, c - lin) + f
+            c = np.einsum("qrbd,rbd->qbd", M, x) + v
+            lin = last
+        return torch.tensor([r], dtype=torch.float64)
 
-    def update(self, carry):
-        c = carry.numpy()
-        Hn = self.P[0] + sum((self.P[1 + j] - self.P[0]) * c[j][:, None, :] for j in range(self.NS))
-        self.res[0] = self._residual(Hn, c)
-        self.H = torch.from_numpy(Hn.copy())
-        self.lin = c.copy()
+    def apply(self, k):
+        Hk = self.H.numpy()
+        Hn = np.empty_like(Hk)
+        prev_k, s = self.lin, self.carry
+        for l in range(self.Ls):
+            J, o = self._map(prev_k, l)
+            s = np.einsum("qrbd,rbd->qbd", J, s) + o
+            Hn[:, :, l] = s
+            prev_k = Hk[:, :, l]
+        prev, r = self.carry, 0.0
+        for l in range(self.Ls):
+            # NaN kept, like the kernels' max.NaN (Python's max would drop it)
+            r = float(np.maximum(r, np.max(np.abs(Hn[:, :, l] - self.step(prev, self.ug[l], self.a)))))
+            prev = Hn[:, :, l]
+        self.H = torch.from_numpy(Hn)
+        self.res = r
+
+    def pass_outcome(self):
+        return torch.tensor([self.res, 0.0], dtype=torch.float64)
 
 
 def _free_port():
