@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         phases ^= 1u << stage;
 
         const int r0 = w * T;
-        Map agg[kV];
+        // the step maps stay in registers for the second sweep
+        Map agg[kV], mt[T][kV];
 #pragma unroll
         for (int j = 0; j < kV; ++j) agg[j] = Map::identity();
 #pragma unroll
@@ -129,7 +130,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
             const int row = r0 + t;
             F4 z4 = load4(sz + row * kDc + lane * kV), c4 = load4(sc + row * kDc + lane * kV);
 #pragma unroll
-            for (int j = 0; j < kV; ++j) agg[j] = compose(linear_gru_map(z4.v[j], c4.v[j]), agg[j]);
+            for (int j = 0; j < kV; ++j) {
+                mt[t][j] = linear_gru_map(z4.v[j], c4.v[j]);
+                agg[j] = compose(mt[t][j], agg[j]);
+            }
         }
         scan_put(scan, w, lane, agg);
         __syncthreads();
@@ -166,13 +170,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         for (int t = 0; t < T; ++t) {
             const int row = r0 + t;
             const long long l = l0 + row;
-            F4 z4 = load4(sz + row * kDc + lane * kV), c4 = load4(sc + row * kDc + lane * kV);
 #pragma unroll
-            for (int j = 0; j < kV; ++j) {
-                const Map m = linear_gru_map(z4.v[j], c4.v[j]);
-                hv[j] = fmaf(m.m, hv[j], m.v);
-            }
-            if (l < L && chv) store4(p.h + ((b * L + l) * D + dch), hv);
+            for (int j = 0; j < kV; ++j) hv[j] = fmaf(mt[t][j].m, hv[j], mt[t][j].v);
+            if (l < L && chv) stcgv<kV>(p.h + ((b * L + l) * D + dch), hv);
         }
         __syncthreads();
         ticket = s_int[6 + (stage ^ 1)];
