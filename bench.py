@@ -344,13 +344,71 @@ def measure(w, dev, stream, reps=10, warmup=3, baselines=True):
     return out
 
 
+def run_projection(dev, stream, B=8, L=4096, Din=1024, D=1024, reps=10):
+    """The ParaGRU solve from the layer input, x [B,L,Din] -> u = x w^T
+    (bf16, fp32 accumulation) -> Newton solve: the fused path (the projection
+    on the tensor cores with pass 0 in its epilogue, pararnn_gru_project_solve)
+    against the projection as a cuBLAS GEMM (torch.matmul) followed by the
+    solve.  Inputs: x ~ N(0,1), w ~ N(0,1/Din), no bias, a ~ U(-0.5,0.5),
+    h0 ~ N(0,0.1)."""
+    import nonlinear_rnn_newton_b200 as P
+    xi = W.make_projection_inputs(B, L, Din, D, seed=0, bias_std=0.0).to(dev)
+    u = torch.empty((B, L, 3, D), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((B, L, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(P.pararnn_gru_project_workspace_size(B, L, D, Din), dtype=torch.uint8, device=dev)
+    u2 = torch.empty_like(u)
+    h2 = torch.empty_like(h)
+    ws2 = torch.empty(P.pararnn_gru_workspace_size(B, L, D), dtype=torch.uint8, device=dev)
+    x2, w2 = xi.x.view(B * L, Din), xi.w.view(3 * D, Din)
+
+    def fused():
+        P.pararnn_gru_project_solve_async(xi.x, xi.w, None, xi.a, xi.h0, u, h, ws, stream=stream)
+
+    def gemm():
+        with torch.cuda.stream(stream):
+            torch.matmul(x2, w2.t(), out=u2.view(B * L, 3 * D))
+
+    def unfused():
+        gemm()
+        P.pararnn_gru_solve_async(u2, xi.a, xi.h0, h2, ws2, stream=stream)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    t_f, t_u, t_g = timed(fused), timed(unfused), timed(gemm)
+    fused()
+    passes = P.pararnn_read_pass_times(ws, stream)
+    rf = P.pararnn_read_result(ws, stream)
+    unfused()
+    ru = P.pararnn_read_result(ws2, stream)
+    flops = 2.0 * B * L * Din * 3 * D
+    return {"workload": f"gru_project_B{B}_L{L}_Din{Din}_D{D}", "fused_ms": t_f, "gemm_then_solve_ms": t_u,
+            "gemm_ms": t_g, "gemm_tflops": flops / (t_g * 1e-3) / 1e12,
+            "fused_pass0_us": passes[0] if passes else None,
+            "fused_pass0_tflops": flops / (passes[0] * 1e-6) / 1e12 if passes else None,
+            "iters": [rf[1], ru[1]], "status": [rf[0], ru[0]],
+            "max_abs_state_diff": float((h - h2).abs().max()),
+            "u_equal_fraction": float((u == u2).float().mean())}
+
+
 def run_configs(headline, dev, stream):
-    """Every solve workload except the headline, one after another."""
+    """Every solve workload except the headline, one after another, and the
+    solve from the layer input (the fused input projection)."""
     out = {}
     for w in (W.GRU, W.LSTM) + W.GRU_SWEEP + (W.LSTM_TRAIN,):
         if w.name == headline.name:
             continue
         out[w.name] = measure(w, dev, stream)
+    pr = run_projection(dev, stream)
+    out[pr["workload"]] = pr
     return out
 
 

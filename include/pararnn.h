@@ -162,6 +162,46 @@ PARARNN_API pararnn_status pararnn_result_to_device(const void* workspace, float
 PARARNN_API pararnn_status pararnn_read_result(const void* workspace, pararnn_stream_t stream,
                                    pararnn_result* result);
 
+/* ------------------------------- input projection fused with Newton pass 0 */
+
+/* ParaGRU solve from the layer input: the gate pre-activations are the input
+ * projection u = x W^T + bias ("O compromisso que SSMs fizeram": the input
+ * enters the recurrence through a projection, B_l x_l), computed on the
+ * tensor cores in a kernel whose epilogue also runs Newton pass 0 ("A
+ * sacada: método de Newton": at the initial guess H^0 = 0 the step maps
+ * depend on the gates alone), so the first pass neither waits for u nor
+ * reads it back.  The solve then continues from H^1 exactly as
+ * pararnn_gru_solve (same stopping rule, status, iteration count).
+ *   x     [B][L][Din] bf16, device (Din a multiple of 8)
+ *   w     [3][D][Din] bf16, device: the projection's rows for gates z, r, c
+ *         (row g*D + d produces u[..][g][d]; the layout of a linear layer's
+ *         weight with 3*D outputs)
+ *   bias  [3][D] fp32 or NULL (zeros)
+ *   a, h0 as pararnn_gru_solve
+ *   u     [B][L][3][D] bf16, device, out: u = bf16(x W^T + bias) with an
+ *         fp32 accumulator, rounded to nearest even; the solve runs on these
+ *         rounded values, so pararnn_gru_solve on u gives the same states
+ *   h     [B][L][D] fp32 out
+ * Workspace: pararnn_gru_project_workspace_size(B, L, D, Din) bytes (0 for
+ * invalid shapes).  Errors as pararnn_gru_solve; Din not a positive multiple
+ * of 8 gives UNSUPPORTED.  The _async form queues the work on `stream`; read
+ * the outcome with pararnn_read_result. */
+PARARNN_API size_t pararnn_gru_project_workspace_size(int64_t B, int64_t L, int64_t D, int64_t Din);
+PARARNN_API pararnn_status pararnn_gru_project_solve(const void* x, const void* w, const float* bias,
+                                                     const float* a, const float* h0, void* u,
+                                                     float* h, int64_t B, int64_t L, int64_t Din,
+                                                     int64_t D, float tol, int max_iters,
+                                                     void* workspace, size_t workspace_bytes,
+                                                     pararnn_stream_t stream, int* iters_out,
+                                                     float* residual_out);
+PARARNN_API pararnn_status pararnn_gru_project_solve_async(const void* x, const void* w,
+                                                           const float* bias, const float* a,
+                                                           const float* h0, void* u, float* h,
+                                                           int64_t B, int64_t L, int64_t Din,
+                                                           int64_t D, float tol, int max_iters,
+                                                           void* workspace, size_t workspace_bytes,
+                                                           pararnn_stream_t stream);
+
 /* ------------------------------------------------- fixed-scratch solve */
 
 /* ParaGRU Newton solve without a caller workspace.  The pages have no

@@ -48,6 +48,9 @@ __all__ = [
     "pararnn_read_pass_times",
     "pararnn_segment_record_floats",
     "pararnn_result_to_device",
+    "pararnn_gru_project_workspace_size",
+    "pararnn_gru_project_solve",
+    "pararnn_gru_project_solve_async",
     "pararnn_segment_fold_workspace_size",
     "pararnn_read_result",
     "pararnn_selftest_wait_timeout",

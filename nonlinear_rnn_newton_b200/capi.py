@@ -91,6 +91,11 @@ SIGNATURES = {
     "pararnn_lstm_segment_pass": (_st, [_vp, _st, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                         ctypes.c_size_t, _vp]),
     "pararnn_result_to_device": (_st, [_vp, _vp, _vp]),
+    "pararnn_gru_project_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
+    "pararnn_gru_project_solve": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_float,
+                                        ctypes.c_int, _vp, ctypes.c_size_t, _vp, _vp, _vp]),
+    "pararnn_gru_project_solve_async": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                              ctypes.c_float, ctypes.c_int, _vp, ctypes.c_size_t, _vp]),
     "pararnn_segment_record_floats": (ctypes.c_size_t, [ctypes.c_int, _i64, _i64]),
     "pararnn_segment_fold_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _i64, _i64, _i64]),
     "pararnn_gru_segment_fold": (_st, [_vp, _st, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
@@ -285,6 +290,63 @@ def pararnn_gru_solve_noalloc(u, a, h0, h, tol=1e-6, max_iters=10, stream=None):
                                            ctypes.byref(it), ctypes.byref(res))
     _check(st)
     return it.value, res.value, st
+
+
+def pararnn_gru_project_workspace_size(B, L, D, Din):
+    return int(lib.pararnn_gru_project_workspace_size(B, L, D, Din))
+
+
+def _project_args(x, w, bias, a, h0, u, h):
+    if x.dim() != 3 or w.dim() != 3:
+        raise ValueError("x must be [B,L,Din] and w [3,D,Din]")
+    B, L, Din = x.shape
+    G, D, Din2 = w.shape
+    if G != 3 or Din2 != Din:
+        raise ValueError(f"w must be [3,D,{Din}], got {tuple(w.shape)}")
+    _need(x, "x", (B, L, Din), dtype=torch.bfloat16, device=x.device)
+    _need(w, "w", (3, D, Din), dtype=torch.bfloat16, device=x.device)
+    _need(bias, "bias", (3, D), device=x.device)
+    _need(a, "a", (3, D), device=x.device)
+    _need(h0, "h0", (B, D), device=x.device)
+    _need(u, "u", (B, L, 3, D), dtype=torch.bfloat16, device=x.device)
+    _need(h, "h", (B, L, D), device=x.device)
+    return B, L, Din, D
+
+
+def pararnn_gru_project_solve(x, w, bias, a, h0=None, tol=1e-6, max_iters=10, u=None, h=None, workspace=None,
+                              stream=None):
+    """ParaGRU solve from the layer input: u = bf16(x w^T + bias) on the tensor
+    cores with Newton pass 0 in the same kernel, then the rest of the solve.
+    x [B,L,Din] bf16, w [3,D,Din] bf16, bias [3,D] fp32 or None (device
+    tensors).  Returns (u [B,L,3,D] bf16, h [B,L,D], iters, residual, status)."""
+    B, L, Din = x.shape
+    D = w.shape[1]
+    dev = x.device
+    if u is None:
+        u = torch.empty((B, L, 3, D), dtype=torch.bfloat16, device=dev)
+    if h is None:
+        h = torch.empty((B, L, D), dtype=torch.float32, device=dev)
+    _project_args(x, w, bias, a, h0, u, h)
+    ws = _workspace(pararnn_gru_project_workspace_size(B, L, D, Din), dev, workspace)
+    it = ctypes.c_int(0)
+    res = ctypes.c_float(0.0)
+    with torch.cuda.device(dev):
+        st = lib.pararnn_gru_project_solve(_ptr(x), _ptr(w), _ptr(bias), _ptr(a), _ptr(h0), _ptr(u), _ptr(h), B, L,
+                                           Din, D, float(tol), int(max_iters), _ptr(ws),
+                                           ws.numel() * ws.element_size(), _stream(dev, stream), ctypes.byref(it),
+                                           ctypes.byref(res))
+    _check(st)
+    return u, h, it.value, res.value, st
+
+
+def pararnn_gru_project_solve_async(x, w, bias, a, h0, u, h, workspace, tol=1e-6, max_iters=10, stream=None):
+    """Queue the fused projection + solve (device tensors only); read the
+    outcome with pararnn_read_result(workspace)."""
+    B, L, Din, D = _project_args(x, w, bias, a, h0, u, h)
+    st = lib.pararnn_gru_project_solve_async(_ptr(x), _ptr(w), _ptr(bias), _ptr(a), _ptr(h0), _ptr(u), _ptr(h), B,
+                                             L, Din, D, float(tol), int(max_iters), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(x.device, stream))
+    return _check(st)
 
 
 def pararnn_gru_solve_noalloc_max_scratch():

@@ -383,6 +383,14 @@ __device__ __forceinline__ float min_keep_nan(float x, float hi)
     return r;
 }
 
+// max(a, b) with NaN kept (either NaN gives NaN)
+__device__ __forceinline__ float max_keep_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 // 1 + e^-x with the exponent clamped (see above)
 __device__ __forceinline__ float logistic_den(float x)
 {

@@ -61,12 +61,6 @@ __host__ __device__ constexpr long long solve_desc_count(int n_chunks, long long
     return (long long)((n_chunks + kGroup - 1) / kGroup) * BS;
 }
 
-__device__ __forceinline__ float max_keep_nan(float a, float b)
-{
-    float r;
-    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-    return r;
-}
 
 // CW: compute warps = row pairs (two steps each) in a tile.
 template <class Cell, class UT, int CW>
@@ -159,9 +153,25 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
         prefetch_tensormap(&tm_bnd);
     }
 
-    if (tid == 0 && blockIdx.x == 0) hdr->t_pass[0] = global_timer_ns();
+    // pass 0 may have run already, fused with the input projection: then the
+    // decision after it comes first (from the residuals that kernel left)
+    const int k0 = hdr->k0;
+    if (tid == 0 && blockIdx.x == 0) hdr->t_pass[k0] = global_timer_ns();
+    if (k0 == 1) {
+        if (tid == 0) {
+            NewtonDecision d = newton_decide(hdr, 0, 0, true, p.tol, p.max_iters);
+            if (!d.cont && blockIdx.x == 0) newton_publish(hdr, d, 0);
+            s_int[2] = d.cont;
+            s_int[3] = d.zero;
+        }
+        __syncthreads();
+        if (!s_int[2]) {
+            if (s_int[3]) newton_zero_states<NS>(p, tid, blockDim.x);
+            return;
+        }
+    }
 
-    for (int k = 0;; ++k) {
+    for (int k = k0;; ++k) {
         const int slot = k % 3;
         const bool first = (k == 0) && !(Seg && hdr->seg_warm);  // the pass starts from H^0 = 0
         if (tid == 0) {
@@ -172,7 +182,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
             }
             // fresh barriers every pass (no copy is in flight between passes)
             for (int i = 0; i < kStages; ++i) {
-                if (k > 0) {
+                if (k > k0) {
                     mbar_inval(&bar_full[i]);
                     mbar_inval(&bar_empty[i]);
                 }
@@ -180,7 +190,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 mbar_init(&bar_empty[i], CWT);
             }
             for (int i = 0; i < kWork; ++i) {
-                if (k > 0) {
+                if (k > k0) {
                     mbar_inval(&bar_aggr[i]);
                     mbar_inval(&bar_carry[i]);
                 }
@@ -704,7 +714,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
             if (first) atomicMax(&hdr->res0, __float_as_uint(b2) & 0x7fffffffu);
         }
 
-        const bool bar_ok = grid_barrier(&hdr->bar, unsigned(k), err, p.wait_ns, &s_int[1]);
+        const bool bar_ok = grid_barrier(&hdr->bar, unsigned(k - k0), err, p.wait_ns, &s_int[1]);
         if (tid == 0) {
             // every CTA has finished pass k
             if (blockIdx.x == 0 && k + 1 < kPassTimes) hdr->t_pass[k + 1] = global_timer_ns();

@@ -24,6 +24,7 @@
 #include "segment.cuh"
 #include "adjoint.cuh"
 #include "linear_scan.cuh"
+#include "project.cuh"
 
 using namespace pararnn;
 
@@ -287,7 +288,8 @@ pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid, int th
 template <class Cell, class UT, int T, bool Seg, int LB>
 pararnn_status launch_newton_k(const Shape& s, const void* u, pararnn_dtype dt, const float* a,
                                const float* const s0[2], float* const st[2], float tol, int max_iters, void* ws,
-                               cudaStream_t stream, const float* const* in, const float* const* slin, int warm)
+                               cudaStream_t stream, const float* const* in, const float* const* slin, int warm,
+                               bool zero_ws)
 {
     constexpr int NS = Cell::NS;
     constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
@@ -298,7 +300,7 @@ pararnn_status launch_newton_k(const Shape& s, const void* u, pararnn_dtype dt, 
     if (s.Lc != KL::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, KL::Lc);
     const ScanLayout ly = scan_layout(s, desc_words, solve_bnd_bytes(s, NS), solve_descs(s));
     unsigned char* wsb = static_cast<unsigned char*>(ws);
-    CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));  // header + descriptors
+    if (zero_ws) CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));  // header + descriptors
 
     CUtensorMap tu, t0, t1;
     TRY(map_gates(&tu, u, dt, Cell::G, Cell::G, s, KL::Lc));
@@ -361,13 +363,16 @@ pararnn_status launch_newton_k(const Shape& s, const void* u, pararnn_dtype dt, 
 template <class Cell, class UT, int T, bool Seg = false>
 pararnn_status launch_newton(const Shape& s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
                              float* const st[2], float tol, int max_iters, void* ws, cudaStream_t stream,
-                             const float* const* in = nullptr, const float* const* slin = nullptr, int warm = 0)
+                             const float* const* in = nullptr, const float* const* slin = nullptr, int warm = 0,
+                             bool zero_ws = true)
 {
     int sms = 0;
     TRY(device_info(&sms));
     if (solve_lookback_walks(std::min(s.n_tiles, sms), s.B * s.S))
-        return launch_newton_k<Cell, UT, T, Seg, 1>(s, u, dt, a, s0, st, tol, max_iters, ws, stream, in, slin, warm);
-    return launch_newton_k<Cell, UT, T, Seg, 0>(s, u, dt, a, s0, st, tol, max_iters, ws, stream, in, slin, warm);
+        return launch_newton_k<Cell, UT, T, Seg, 1>(s, u, dt, a, s0, st, tol, max_iters, ws, stream, in, slin, warm,
+                                                    zero_ws);
+    return launch_newton_k<Cell, UT, T, Seg, 0>(s, u, dt, a, s0, st, tol, max_iters, ws, stream, in, slin, warm,
+                                                zero_ws);
 }
 
 size_t solve_ws_bytes(int cell, long long B, long long L, long long D)
@@ -612,6 +617,106 @@ pararnn_status finish_sync(void* ws, cudaStream_t stream, int* iters_out, float*
     if (iters_out) *iters_out = r.iters;
     if (residual_out) *residual_out = r.residual;
     return st;
+}
+
+// ------------------------------------- input projection fused with pass 0
+
+// bf16 [n2][n1][n0] (n0 contiguous) -> box {64, rows, 1} with the 128-byte
+// swizzle the tensor-core operand descriptors expect.
+pararnn_status map_bf16_sw128(CUtensorMap* m, const void* p, cuuint64_t n0, cuuint64_t n1, cuuint64_t n2,
+                              cuuint32_t rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {n0, n1, n2};
+    cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+    cuuint32_t box[3] = {cuuint32_t(kPK), rows, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PARARNN_ERR_CUDA, "cuTensorMapEncodeTiled(projection operand) failed: %d", int(r));
+    return PARARNN_OK;
+}
+
+long long project_tiles(long long B, long long L, long long D)
+{
+    return ((L + kPM - 1) / kPM) * B * ((D + kPC - 1) / kPC);
+}
+
+// the solve's workspace, then the fused kernel's look-back descriptors
+size_t project_ws_bytes(long long B, long long L, long long D, long long Din)
+{
+    if (!shape_ok(B, L, D) || D % 8 != 0 || Din < 8 || Din % 8 != 0) return 0;
+    const size_t solve = solve_ws_bytes(0, B, L, D);
+    if (!solve) return 0;
+    return align256(solve + size_t(project_tiles(B, L, D)) * kPDescWords * 8);
+}
+
+pararnn_status project_solve_async(const void* x, const void* w, const float* bias, const float* a, const float* h0,
+                                   uint16_t* u, float* h, long long B, long long L, long long Din, long long D,
+                                   float tol, int max_iters, void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    t_err[0] = '\0';
+    TRY(check_ptr(x, "x", true));
+    TRY(check_ptr(w, "w", true));
+    TRY(check_ptr(bias, "bias", false));
+    TRY(check_ptr(u, "u", true));
+    TRY(solve_args(0, u, PARARNN_BF16, a, nullptr, h0, nullptr, h, B, L, D, tol, max_iters));
+    if (Din < 8 || Din % 8 != 0) return fail(PARARNN_ERR_UNSUPPORTED, "Din must be a positive multiple of 8 (got %lld)", Din);
+    if ((double)B * (double)L * (double)Din * 2.0 >= 1099511627776.0) return fail(PARARNN_ERR_INVALID_ARG, "x too large");
+    if (project_tiles(B, L, D) > INT_MAX / 2) return fail(PARARNN_ERR_INVALID_ARG, "too many tiles");
+    TRY(check_workspace(ws, ws_bytes, project_ws_bytes(B, L, D, Din)));
+    Shape s;
+    TRY(make_shape(B, L, D, gru_lc<uint16_t>(), &s));
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    const size_t solve = solve_ws_bytes(0, B, L, D);
+    const long long nt = project_tiles(B, L, D);
+    const ScanLayout ly = scan_layout(s, TileDesc<Aff<1>, 1>::words, solve_bnd_bytes(s, 1), solve_descs(s));
+    CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));  // header + the solve's descriptors
+    CUDA_TRY(cudaMemsetAsync(wsb + solve, 0, size_t(nt) * kPDescWords * 8, stream));
+
+    CUtensorMap tx, tw;
+    TRY(map_bf16_sw128(&tx, x, cuuint64_t(Din), cuuint64_t(L), cuuint64_t(B), kPM));
+    TRY(map_bf16_sw128(&tw, w, cuuint64_t(Din), cuuint64_t(D), 3, kPC));
+    ProjectParams p;
+    p.bias = bias;
+    p.a = a;
+    p.h0 = h0;
+    p.u = u;
+    p.h = h;
+    p.B = B;
+    p.L = L;
+    p.D = D;
+    p.Din = Din;
+    p.Sf = int((D + kPC - 1) / kPC);
+    p.n_chunks = int((L + kPM - 1) / kPM);
+    p.n_tiles = int(nt);
+    p.hdr = reinterpret_cast<WsHeader*>(wsb);
+    p.desc = reinterpret_cast<unsigned long long*>(wsb + solve);
+    p.wait_ns = kWaitLimitNs;
+    using PL = ProjectLayout<3>;
+    CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(project_pass0_kernel),
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, int(PL::smem_bytes)));
+    project_pass0_kernel<<<unsigned(nt), 128, PL::smem_bytes, stream>>>(tx, tw, p);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+
+    // H^1 at the solve's chunk ends into the boundary rows pass 1 reads
+    // (ring slot 1), then the fused solve from pass 1 on the same header
+    float* bnd = reinterpret_cast<float*>(wsb + ly.extra);
+    if (s.n_chunks > 1) {
+        const long long n = (long long)s.B * (s.n_chunks - 1) * (s.D / 4);
+        bnd_gather_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(h, h, bnd + size_t(s.B) * s.n_chunks * s.S * kDc,
+                                                                          1, s.B, s.L, s.D, s.n_chunks, s.Lc,
+                                                                          s.S * kDc);
+        CUDA_TRY(cudaGetLastError());
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+    const float* s0[2] = {h0, nullptr};
+    float* st[2] = {h, nullptr};
+    return launch_newton<GruCell, uint16_t, gru_tile_arg<uint16_t>()>(s, u, PARARNN_BF16, a, s0, st, tol, max_iters,
+                                                                      ws, stream, nullptr, nullptr, 0, false);
 }
 
 // --------------------------------------------------------------- adjoints
@@ -943,6 +1048,31 @@ pararnn_status pararnn_gru_solve_noalloc(const void* u, pararnn_dtype u_dtype, c
 }
 
 size_t pararnn_gru_solve_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
+
+size_t pararnn_gru_project_workspace_size(int64_t B, int64_t L, int64_t D, int64_t Din)
+{
+    return project_ws_bytes(B, L, D, Din);
+}
+
+pararnn_status pararnn_gru_project_solve_async(const void* x, const void* w, const float* bias, const float* a,
+                                               const float* h0, void* u, float* h, int64_t B, int64_t L,
+                                               int64_t Din, int64_t D, float tol, int max_iters, void* workspace,
+                                               size_t workspace_bytes, pararnn_stream_t stream)
+{
+    return project_solve_async(x, w, bias, a, h0, static_cast<uint16_t*>(u), h, B, L, Din, D, tol, max_iters,
+                               workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pararnn_status pararnn_gru_project_solve(const void* x, const void* w, const float* bias, const float* a,
+                                         const float* h0, void* u, float* h, int64_t B, int64_t L, int64_t Din,
+                                         int64_t D, float tol, int max_iters, void* workspace,
+                                         size_t workspace_bytes, pararnn_stream_t stream, int* iters_out,
+                                         float* residual_out)
+{
+    TRY(pararnn_gru_project_solve_async(x, w, bias, a, h0, u, h, B, L, Din, D, tol, max_iters, workspace,
+                                        workspace_bytes, stream));
+    return finish_sync(workspace, reinterpret_cast<cudaStream_t>(stream), iters_out, residual_out);
+}
 
 pararnn_status pararnn_lstm_solve_async(const void* u, pararnn_dtype u_dtype, const float* a, const float* c0,
                                         const float* h0, float* c, float* h, int64_t B, int64_t L, int64_t D,

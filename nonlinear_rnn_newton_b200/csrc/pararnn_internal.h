@@ -46,7 +46,11 @@ struct alignas(256) WsHeader {
     // the zero guess (0).
     unsigned long long seg_lin[2];
     int seg_warm;
-    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result) - 8 * kPassTimes - 8 * 2 - 4];
+    // The pass the fused solve starts with: 0, or 1 when pass 0 ran in the
+    // projection kernel (which then left H^1, the residuals of H^0 and H^1
+    // in res0 and res[0], and its own ticket count in tick[3]).
+    int k0;
+    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result) - 8 * kPassTimes - 8 * 2 - 4 - 4];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
 

@@ -102,3 +102,33 @@ def make_inputs(w: Workload, seed: int = 0, a_scale: float = 1.0) -> Inputs:
     if w.train:
         dh = torch.randn((w.B, w.L, w.D), generator=g, dtype=torch.float32)
     return Inputs(u=u, a=a, h0=h0, c0=c0, dh=dh)
+
+
+@dataclass
+class ProjectionInputs:
+    x: torch.Tensor                 # [B,L,Din] bfloat16
+    w: torch.Tensor                 # [3,D,Din] bfloat16
+    bias: Optional[torch.Tensor]    # [3,D] float32 or None
+    a: torch.Tensor                 # [3,D] float32
+    h0: Optional[torch.Tensor]      # [B,D] float32 or None
+
+    def to(self, device):
+        mv = lambda t: None if t is None else t.to(device)
+        return ProjectionInputs(mv(self.x), mv(self.w), mv(self.bias), mv(self.a), mv(self.h0))
+
+
+def make_projection_inputs(B: int, L: int, Din: int, D: int, seed: int = 0, h0_std: float = 0.1,
+                           bias_std: float = 0.1) -> ProjectionInputs:
+    """Inputs of the ParaGRU layer fed through its input projection, drawn on
+    the CPU in the order x, w, bias, a, h0: x ~ N(0,1) and w ~ N(0, 1/Din),
+    both rounded to bfloat16, so that the gate pre-activations x w^T are
+    about N(0,1) like the solve workloads' u; bias ~ N(0, bias_std) (None if
+    0); a ~ U(-0.5,0.5); h0 ~ N(0, h0_std) (None if 0)."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((B, L, Din), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    w = (torch.randn((3, D, Din), generator=g, dtype=torch.float32) / Din ** 0.5).to(torch.bfloat16)
+    bias = torch.randn((3, D), generator=g, dtype=torch.float32) * bias_std if bias_std > 0 else None
+    a = torch.rand((3, D), generator=g, dtype=torch.float32) - 0.5
+    h0 = torch.randn((B, D), generator=g, dtype=torch.float32) * h0_std if h0_std > 0 else None
+    return ProjectionInputs(x, w, bias, a, h0)
+

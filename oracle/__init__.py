@@ -176,5 +176,19 @@ def lstm_bptt(u, a, c0, h0, gh, gc=None):
     return du, da, dc0, dh0
 
 
+def project(x, w, bias=None):
+    """Input projection of the gate pre-activations in float64:
+    u[b, l, g, d] = sum_k x[b, l, k] w[g, d, k] + bias[g, d]
+    (x [B, L, Din], w [G, D, Din], bias [G, D] or None).  Page "ParaRNN: Apple
+    destrava treino paralelo de RNNs não-lineares e escala pra 7B parâmetros",
+    section "O compromisso que SSMs fizeram": the input enters the recurrence
+    through a projection (B_l x_l).  A library contraction is the step."""
+    x, w = _f64(x), _f64(w)
+    u = np.einsum("blk,gdk->blgd", x, w)
+    if bias is not None:
+        u = u + _f64(bias)[None, None]
+    return u
+
+
 def library_path() -> str:
     return os.path.abspath(_build.LIB)

@@ -406,3 +406,38 @@ def test_regression_fixture_unchanged():
     assert it == g["iters"] and st == g["status"]
     for b, l, d, vc, vh in g["samples"]:
         assert abs(c[b, l, d] - vc) < 1e-13 and abs(h[b, l, d] - vh) < 1e-13
+
+
+# ------------------------------------------------------- input projection
+
+def test_projection_matches_brute_force_sum():
+    """oracle.project against the definition summed term by term in Python."""
+    g = torch.Generator().manual_seed(11)
+    B, L, Din, G, D = 2, 3, 5, 3, 2
+    x = torch.randn((B, L, Din), generator=g, dtype=torch.float64)
+    w = torch.randn((G, D, Din), generator=g, dtype=torch.float64)
+    bias = torch.randn((G, D), generator=g, dtype=torch.float64)
+    u = oracle.project(x, w, bias)
+    for b in range(B):
+        for l in range(L):
+            for gg in range(G):
+                for d in range(D):
+                    ref = float(bias[gg, d])
+                    for k in range(Din):
+                        ref += float(x[b, l, k]) * float(w[gg, d, k])
+                    assert abs(u[b, l, gg, d] - ref) < 1e-12
+
+
+def test_projection_special_cases():
+    """Identity weights give x + bias (the weight row g*D+d picks input g*D+d);
+    zero input gives the bias."""
+    g = torch.Generator().manual_seed(12)
+    B, L, G, D = 2, 4, 3, 5
+    x = torch.randn((B, L, G * D), generator=g, dtype=torch.float64)
+    bias = torch.randn((G, D), generator=g, dtype=torch.float64)
+    eye = torch.eye(G * D, dtype=torch.float64).reshape(G, D, G * D)
+    u = oracle.project(x, eye, bias)
+    np.testing.assert_allclose(u, (x.reshape(B, L, G, D) + bias).numpy(), rtol=0, atol=1e-15)
+    z = oracle.project(torch.zeros((B, L, 7), dtype=torch.float64), torch.randn((G, D, 7), generator=g,
+                                                                                dtype=torch.float64), bias)
+    np.testing.assert_array_equal(z, np.broadcast_to(bias.numpy(), (B, L, G, D)))
