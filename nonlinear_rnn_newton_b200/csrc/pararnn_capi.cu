@@ -696,10 +696,11 @@ pararnn_status project_solve_async(const void* x, const void* w, const float* bi
     p.desc = reinterpret_cast<unsigned long long*>(wsb + solve);
     p.wait_ns = kWaitLimitNs;
     using PL = ProjectLayout<3>;
-    CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(project_pass0_kernel),
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, int(PL::smem_bytes)));
-    project_pass0_kernel<<<unsigned(nt), 128, PL::smem_bytes, stream>>>(tx, tw, p);
-    CUDA_TRY(cudaGetLastError());
+    int grid = 0;
+    TRY(resident_grid(project_pass0_kernel, PL::smem_bytes, int(nt), &grid, kPThreads));
+    void* args[] = {(void*)&tx, (void*)&tw, (void*)&p};
+    CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(project_pass0_kernel), dim3(grid),
+                                         dim3(kPThreads), args, PL::smem_bytes, stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
 
     // H^1 at the solve's chunk ends into the boundary rows pass 1 reads
