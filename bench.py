@@ -712,12 +712,19 @@ def main():
     ap.add_argument("--cells", action="store_true", help="add the runtime-compiled user cells (GRU, LSTM sources)")
     ap.add_argument("--seq-segments", default="", help="comma list of R: the solve with each sequence split into "
                     "R segments (sequence sharding), run on this GPU one segment after another")
+    ap.add_argument("--projection-only", action="store_true", help="only the solve from the layer input (fused "
+                    "input projection against cuBLAS GEMM + solve), one JSON object; for profiling")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.BY_NAME[args.workload]
 
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.projection_only:
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_projection(dev, torch.cuda.Stream(dev), reps=args.steps)), flush=True)
         return
 
     rank, world, local = dist_setup()
