@@ -23,6 +23,7 @@
 #include "decode.cuh"
 #include "segment.cuh"
 #include "adjoint.cuh"
+#include "adjoint_ws.cuh"
 #include "linear_scan.cuh"
 #include "project.cuh"
 
@@ -722,37 +723,47 @@ pararnn_status project_solve_async(const void* x, const void* w, const float* bi
 
 // --------------------------------------------------------------- adjoints
 
+// Compute warps (two steps each) of the warp-specialised adjoint per cell and
+// gate dtype; fp32 gates need twice the staging space, so their tiles are half
+// as long.
+template <class Cell, class UT> constexpr int adj_warps()
+{
+    return (Cell::NS == 1 ? 11 : 7) / (sizeof(UT) == 2 ? 1 : 2);
+}
+// workspace sizing uses the shortest tile (most tiles) of either gate dtype
+template <class Cell> constexpr int adj_lc_min() { return 2 * adj_warps<Cell, float>(); }
+
 size_t adjoint_ws_bytes(int cell, long long B, long long L, long long D)
 {
     if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
     Shape s;
     char saved[sizeof(t_err)];
     memcpy(saved, t_err, sizeof(t_err));
-    pararnn_status st = make_shape(B, L, D, kLcAdj, &s);
+    pararnn_status st = make_shape(B, L, D, cell == 0 ? adj_lc_min<GruCell>() : adj_lc_min<LstmCell>(), &s);
     memcpy(t_err, saved, sizeof(t_err));
     if (st != PARARNN_OK) return 0;
     const int G = cell == 0 ? 3 : 4;
-    const int desc = cell == 0 ? AdjointLayout<GruCell, float, kLcAdj / kWarps>::desc_words
-                               : AdjointLayout<LstmCell, float, kLcAdj / kWarps>::desc_words;
+    const int desc = cell == 0 ? TileDesc<Aff<1>, 1>::words : TileDesc<Aff<2>, 2>::words;
     return scan_layout(s, desc, size_t(s.n_tiles) * G * kDc * 4).total;
 }
 
-template <class Cell, class UT, int T>
-pararnn_status launch_adjoint(const Shape& s, const void* u, pararnn_dtype dt, const float* a,
-                              const float* const s0[2], const float* const st[2], const float* const g[2],
-                              float* du, float* da, float* const ds0[2], void* ws, cudaStream_t stream)
+template <class Cell, class UT>
+pararnn_status launch_adjoint(Shape s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
+                              const float* const st[2], const float* const g[2], float* du, float* da,
+                              float* const ds0[2], void* ws, cudaStream_t stream)
 {
-    using LY = AdjointLayout<Cell, UT, T>;
+    constexpr int CW = adj_warps<Cell, UT>();
+    using LY = AdjointWsLayout<Cell, UT, CW>;
     constexpr int NS = Cell::NS, G = Cell::G;
+    TRY(make_shape(s.B, s.L, s.D, LY::Lc, &s));
     const ScanLayout ly = scan_layout(s, LY::desc_words, size_t(s.n_tiles) * G * kDc * 4);
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));
 
     CUtensorMap tu, t0, t1, tg0, tg1;
-    if (s.Lc != LY::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, LY::Lc);
     TRY(map_gates(&tu, u, dt, G, G, s, LY::Lc));
-    TRY(map_state(&t0, st[0], s, LY::Lc));
-    TRY(map_state(&t1, st[NS - 1], s, LY::Lc));
+    TRY(map_state(&t0, st[0], s, LY::Lc + 1));  // from the row before the tile
+    TRY(map_state(&t1, st[NS - 1], s, LY::Lc + 1));
     const float* gfirst = g[0] ? g[0] : g[NS - 1];
     TRY(map_state(&tg0, gfirst, s, LY::Lc));
     TRY(map_state(&tg1, g[NS - 1], s, LY::Lc));
@@ -779,10 +790,10 @@ pararnn_status launch_adjoint(const Shape& s, const void* u, pararnn_dtype dt, c
     p.partial = reinterpret_cast<float*>(wsb + ly.extra);
     p.wait_ns = kWaitLimitNs;
 
-    auto kern = adjoint_kernel<Cell, UT, T>;
+    auto kern = adjoint_ws_kernel<Cell, UT, CW>;
     int grid = 0;
-    TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid));
-    kern<<<grid, kThreads, LY::smem_bytes, stream>>>(tu, t0, t1, tg0, tg1, p);
+    TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid, LY::threads));
+    kern<<<grid, LY::threads, LY::smem_bytes, stream>>>(tu, t0, t1, tg0, tg1, p);
     CUDA_TRY(cudaGetLastError());
     const long long GD = (long long)G * s.D;
     da_reduce_kernel<<<unsigned((GD + 31) / 32), 256, 0, stream>>>(p.partial, da, int(s.B) * s.n_chunks, s.S, G, s.D);
@@ -821,16 +832,16 @@ pararnn_status adjoint_async(int cell, const void* u, pararnn_dtype dt, const fl
         const float* g[2] = {dh, nullptr};
         float* ds0[2] = {dh0, nullptr};
         if (dt == PARARNN_BF16)
-            return launch_adjoint<GruCell, uint16_t, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
-        return launch_adjoint<GruCell, float, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+            return launch_adjoint<GruCell, uint16_t>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+        return launch_adjoint<GruCell, float>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
     }
     const float* s0[2] = {c0, h0};
     const float* st[2] = {c, h};
     const float* g[2] = {dc, dh};
     float* ds0[2] = {dc0, dh0};
     if (dt == PARARNN_BF16)
-        return launch_adjoint<LstmCell, uint16_t, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
-    return launch_adjoint<LstmCell, float, kLcAdj / kWarps>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+        return launch_adjoint<LstmCell, uint16_t>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+    return launch_adjoint<LstmCell, float>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
 }
 
 // ------------------------------------------------------------ linear scan
