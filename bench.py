@@ -94,18 +94,28 @@ def adjoint_bytes(w: W.Workload) -> int:
     return w.N * (w.G * es + ns * 4 + 4 + w.G * 4)
 
 
-def source_digest() -> str:
+# the sources each profiled kernel is compiled from (its device code)
+_COMMON = ["device_common.cuh", "pararnn_internal.h", "cells.cuh", "scan_common.cuh"]
+KERNEL_SOURCES = {
+    "newton_solve_ws_kernel": _COMMON + ["newton.cuh", "newton_ws.cuh"],
+    "adjoint_kernel": _COMMON + ["adjoint.cuh", "adjoint_ws.cuh"],
+    "project_pass0_kernel": _COMMON + ["project.cuh"],
+}
+
+
+def source_digest(kernel: str) -> str:
+    """Digest of the device sources of `kernel`; a profile summary records it,
+    so that its counters are used only while the kernel is unchanged."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
 def profile_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
-    workload, or None when there is none or the kernel sources changed since
+    workload, or None when there is none or the kernel's sources changed since
     the counters were taken."""
     path = os.path.join(PROFILES, f"{kernel}__{workload}.md")
     try:
@@ -114,7 +124,7 @@ def profile_traffic(kernel: str, workload: str):
         return None
     m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
     m_s = re.search(r"^source_digest:\s*([0-9a-f]+)", text, re.M)
-    if not m_t or not m_s or m_s.group(1) != source_digest():
+    if not m_t or not m_s or m_s.group(1) != source_digest(kernel):
         return None
     return int(m_t.group(1))
 
