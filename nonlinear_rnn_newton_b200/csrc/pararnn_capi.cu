@@ -59,9 +59,6 @@ pararnn_status fail(pararnn_status s, const char* fmt, ...)
 #ifndef PARARNN_ADJ_ROWS
 #define PARARNN_ADJ_ROWS 4
 #endif
-#ifndef PARARNN_LIN_ROWS
-#define PARARNN_LIN_ROWS 8
-#endif
 constexpr size_t kSelftestWorkspace = 16384;
 #ifndef PARARNN_WS_GRU_WARPS
 #define PARARNN_WS_GRU_WARPS 15
@@ -79,7 +76,6 @@ template <class UT> constexpr int lstm_lc() { return 2 * lstm_tile_arg<UT>(); }
 constexpr int kLcGru = gru_lc<float>() < gru_lc<uint16_t>() ? gru_lc<float>() : gru_lc<uint16_t>();
 constexpr int kLcLstm = lstm_lc<float>() < lstm_lc<uint16_t>() ? lstm_lc<float>() : lstm_lc<uint16_t>();
 constexpr int kLcAdj = kWarps * PARARNN_ADJ_ROWS;    // adjoints
-constexpr int kLcLin = kWarps * PARARNN_LIN_ROWS;    // linear scan
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -846,29 +842,50 @@ pararnn_status adjoint_async(int cell, const void* u, pararnn_dtype dt, const fl
 
 // ------------------------------------------------------------ linear scan
 
+// bf16 gates: 15 compute warps of 4 steps (60-step tiles; with the control
+// warp, 16 warps of up to 128 registers); fp32 gates take
+// twice the staging space, so their warps take 2 steps
+#ifndef PARARNN_LIN_CW
+#define PARARNN_LIN_CW 15
+#endif
+constexpr int kLinWarps = PARARNN_LIN_CW;
+template <class UT> constexpr int lin_rows() { return sizeof(UT) == 2 ? 4 : 2; }
+template <class UT> constexpr int lin_lc() { return kLinWarps * lin_rows<UT>(); }
+
 size_t linear_scan_ws_bytes(long long B, long long L, long long D)
 {
     if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
     Shape s;
     char saved[sizeof(t_err)];
     memcpy(saved, t_err, sizeof(t_err));
-    pararnn_status st = make_shape(B, L, D, kLcLin, &s);
+    pararnn_status st = make_shape(B, L, D, lin_lc<float>(), &s);  // the shorter tile: more groups
     memcpy(t_err, saved, sizeof(t_err));
     if (st != PARARNN_OK) return 0;
-    return scan_layout(s, LinScanLayout<float, kLcLin / kWarps>::desc_words, 0).total;
+    return scan_layout(s, LinScanLayout<float, kLinWarps, lin_rows<float>()>::desc_words, 0, solve_descs(s)).total;
 }
 
-template <class UT, int T>
-pararnn_status launch_linear_scan(const Shape& s, const void* u, pararnn_dtype dt, const float* h0, float* h, void* ws,
-                                  cudaStream_t stream)
+// Whether the linear scan's look-backs step back over aggregates.
+#ifndef PARARNN_LIN_WALK
+#define PARARNN_LIN_WALK -1  // -1: chosen from the shape
+#endif
+int linear_scan_walks(int grid, long long sequences)
 {
-    using LY = LinScanLayout<UT, T>;
-    const ScanLayout ly = scan_layout(s, LY::desc_words, 0);
+    return PARARNN_LIN_WALK >= 0 ? PARARNN_LIN_WALK : solve_lookback_walks(grid, sequences);
+}
+
+template <class UT>
+pararnn_status launch_linear_scan(const void* u, pararnn_dtype dt, const float* h0, float* h, long long B,
+                                  long long L, long long D, void* ws, cudaStream_t stream)
+{
+    constexpr int R = lin_rows<UT>();
+    using LY = LinScanLayout<UT, kLinWarps, R>;
+    Shape s;
+    TRY(make_shape(B, L, D, LY::Lc, &s));
+    const ScanLayout ly = scan_layout(s, LY::desc_words, 0, solve_descs(s));
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));
-    CUtensorMap tu1;
-    if (s.Lc != LY::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, LY::Lc);
-    TRY(map_gates(&tu1, u, dt, 3, 1, s, LY::Lc));
+    CUtensorMap tu;
+    TRY(map_gates(&tu, u, dt, 3, 1, s, LY::Lc));
     LinScanParams p;
     p.h0 = h0;
     p.h = h;
@@ -881,10 +898,11 @@ pararnn_status launch_linear_scan(const Shape& s, const void* u, pararnn_dtype d
     p.hdr = reinterpret_cast<WsHeader*>(wsb);
     p.desc = reinterpret_cast<unsigned long long*>(wsb + ly.desc);
     p.wait_ns = kWaitLimitNs;
-    auto kern = linear_scan_kernel<UT, T>;
+    auto kern = linear_scan_kernel<UT, kLinWarps, R>;
     int grid = 0;
-    TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid));
-    kern<<<grid, kThreads, LY::smem_bytes, stream>>>(tu1, p);
+    TRY(resident_grid(kern, LY::smem_bytes, int(solve_descs(s)), &grid, LY::threads));
+    p.lb_walk = linear_scan_walks(grid, s.B * s.S);
+    kern<<<grid, LY::threads, LY::smem_bytes, stream>>>(tu, p);
     CUDA_TRY(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return PARARNN_OK;
@@ -899,10 +917,10 @@ pararnn_status linear_scan_async(const void* u, pararnn_dtype dt, const float* h
     TRY(check_ptr(h0, "h0", false));
     TRY(check_ptr(h, "h", true));
     Shape s;
-    TRY(make_shape(B, L, D, kLcLin, &s));
+    TRY(make_shape(B, L, D, lin_lc<float>(), &s));
     TRY(check_workspace(ws, ws_bytes, linear_scan_ws_bytes(B, L, D)));
-    if (dt == PARARNN_BF16) return launch_linear_scan<uint16_t, kLcLin / kWarps>(s, u, dt, h0, h, ws, stream);
-    return launch_linear_scan<float, kLcLin / kWarps>(s, u, dt, h0, h, ws, stream);
+    if (dt == PARARNN_BF16) return launch_linear_scan<uint16_t>(u, dt, h0, h, B, L, D, ws, stream);
+    return launch_linear_scan<float>(u, dt, h0, h, B, L, D, ws, stream);
 }
 
 // -------------------------------------------------------------- self tests

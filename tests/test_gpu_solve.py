@@ -226,10 +226,14 @@ def test_sequential_baselines_match_oracle(cuda):
     assert H.max_abs(c.cpu().numpy(), cs) <= TOL_STATE and H.max_abs(h.cpu().numpy(), hs) <= TOL_STATE
 
 
-@pytest.mark.parametrize("shape", [(2, 1000, 200), (1, 64, 128), (3, 1, 8)])
-def test_linear_scan_matches_zero_weight_oracle(cuda, shape):
+# (2, 1000, 200): groups of one sequence step back over aggregates (few
+# sequences), ragged tail and slab; (40, 300, 128): many sequences, so
+# look-backs wait for inclusive values; fp32: the shorter tile
+@pytest.mark.parametrize("shape,dt", [((2, 1000, 200), "bf16"), ((1, 64, 128), "bf16"), ((3, 1, 8), "bf16"),
+                                      ((40, 300, 128), "bf16"), ((2, 777, 136), "f32")])
+def test_linear_scan_matches_zero_weight_oracle(cuda, shape, dt):
     B, L, D = shape
-    w = W.custom("gru", B, L, D, "bf16", h0_std=0.1)
+    w = W.custom("gru", B, L, D, dt, h0_std=0.1)
     x = W.make_inputs(w, seed=17)
     xd = x.to(cuda)
     h = P().pararnn_linear_scan(xd.u, xd.h0).cpu().double().numpy()
