@@ -144,18 +144,15 @@ __global__ void __launch_bounds__(32 * (CW + 1), CW < 8 ? 2 : 1)
             }
         };
         // the next tile (ticket, chunk, batch row, first channel): the rest
-        // of the current group, then a new group.  Group tickets are fetched
-        // one group ahead, so that the atomic's round trip overlaps the
-        // current group's work; the divisions are taken once per group
-        // (lane 0 only).
+        // of the current group, then a new group (a group ticket is taken only
+        // when its first tile is issued); the divisions are taken once per
+        // group (lane 0 only).
         const int n_groups = ((p.n_chunks + kGroup - 1) / kGroup) * BS;
-        int g_c = 0, g_end = 0, g_q = 0, g_b = 0, g_d0 = 0, g_next = 0;
-        if (lane == 0) g_next = int(atomicAdd(&hdr->tick[0], 1u));
+        int g_c = 0, g_end = 0, g_q = 0, g_b = 0, g_d0 = 0;
         auto next_tile = [&]() {
             if (g_c >= g_end) {
-                const int gt = g_next;
+                const int gt = int(atomicAdd(&hdr->tick[0], 1u));
                 if (gt >= n_groups) return make_int4(INT_MAX, 0, 0, 0);
-                g_next = int(atomicAdd(&hdr->tick[0], 1u));
                 const int gc = gt / BS;
                 g_q = gt - gc * BS;
                 g_c = gc * kGroup;
