@@ -64,6 +64,13 @@ struct AdjointWsLayout {
     static constexpr bool fits = smem_bytes <= 232448;
 };
 
+// named barrier 1 over the compute warps only
+template <int CW>
+__device__ __forceinline__ void compute_sync_n()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * CW) : "memory");
+}
+
 template <class Cell, class UT, int CW>
 __global__ void __launch_bounds__(32 * (CW + 1), 1)
     adjoint_ws_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_s0,

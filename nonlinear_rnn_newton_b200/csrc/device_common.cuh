@@ -183,14 +183,6 @@ __device__ __forceinline__ void raise_error(int* err, int code)
     atomicCAS(err, 0, code);
 }
 
-// Named barrier 1 over the first CW warps of a CTA (the compute warps of the
-// warp-specialised kernels; the control warp does not take part).
-template <int CW>
-__device__ __forceinline__ void compute_sync_n()
-{
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * CW) : "memory");
-}
-
 __device__ __forceinline__ bool error_raised(const int* err)
 {
     return ld_relaxed_gpu(err) != 0;
