@@ -11,10 +11,10 @@
 // M=128, N=64G, K=Din product), are computed on the tensor cores: a TMA warp
 // brings 64-wide K slices of x and W (128-byte swizzle) into a four-stage
 // shared-memory ring, one thread issues tcgen05.mma (bf16 in, fp32
-// accumulator in tensor memory) and tcgen05.commit releases each stage.  Four
-// epilogue warps read the accumulator (one timestep per thread), add the
-// bias, round to bf16, write u for the later passes, and run Newton pass 0 on
-// the tile: the step maps at H^0, their fold per quarter of the tile, a
+// accumulator in tensor memory) and tcgen05.commit releases each stage.
+// Sixteen epilogue warps read the accumulator (one timestep per thread), add
+// the bias, round to bf16 into shared memory, write u for the later passes
+// from there in whole 128-byte lines, and run Newton pass 0 on the tile: the step maps at H^0, their fold per quarter of the tile, a
 // decoupled look-back along the sequence, the new states H^1 and the
 // residuals of H^0 and H^1.  Two accumulators let the next tile's products
 // run during this tile's epilogue.  The fused solve continues from H^1 with
@@ -145,10 +145,13 @@ struct ProjectLayout {
     static constexpr size_t b_bytes = size_t(G) * kPC * kPK * 2;    // 8 KB per gate
     static constexpr size_t stage_bytes = a_bytes + b_bytes;
     static constexpr size_t ring_bytes = kStages * stage_bytes;
-    // the rounded gates of the tile in the epilogue, [kPM][su_row]
-    static constexpr int su_row = G * kPC * 2 + 16;                 // bytes per timestep (padded)
+    // the rounded gates of the tile in the epilogue, by pairs of timesteps:
+    // [kPM / 2][G][kPC] words, each holding the bf16 gate of timesteps 2i (low
+    // half) and 2i + 1 (high half); rows padded so that the 16-byte writes of
+    // eight consecutive timesteps fall in distinct banks
+    static constexpr int su_row = G * kPC * 4 + 32;                 // bytes per pair of timesteps
     static constexpr size_t off_su = ring_bytes;
-    static constexpr size_t off_misc = off_su + size_t(kPM) * su_row;
+    static constexpr size_t off_misc = off_su + size_t(kPM / 2) * su_row;
     // misc: full[S], empty[S], tmem_full[2], tmem_empty[2]; TMEM address;
     // flags; row-group folds [kPRowGroups][kPC][2]; carry [kPC]; bias
     // [G][kPC]; maxima [2][kPEpiWarps]
@@ -314,36 +317,54 @@ __global__ void __launch_bounds__(kPThreads, 1)
             tc_fence_after();
             epi_sync();  // the bias of this tile is in place; the last tile's gates are read
 
-            // ---- accumulator -> bf16 gates (u in global memory and su)
+            // ---- accumulator -> bf16 gates in su (a thread holds one
+            // timestep; its tensor-memory reads are issued three at a time
+            // before one wait)
             {
                 const int trow = 32 * lq + lane;
-                const long long l = l0 + trow;
                 const uint32_t ta = tmem + uint32_t(acc) * kAccCols + (uint32_t(32 * lq) << 16);
                 constexpr int kChunks = G * kPC / 8 / 4;  // 8-column chunks per column quarter
+                constexpr int kBatch = 3;
+                static_assert(kChunks % kBatch == 0, "chunk batches");
 #pragma unroll
-                for (int k = 0; k < kChunks; ++k) {
-                    const int ch = cq * kChunks + k;       // 8-column chunk of the accumulator
-                    const int g = ch / (kPC / 8), c8 = (ch - g * (kPC / 8)) * 8;
-                    float v[8];
-                    tmem_ld8(ta + uint32_t(g * kPC + c8), v);
+                for (int k0 = 0; k0 < kChunks; k0 += kBatch) {
+                    float v[kBatch][8];
+#pragma unroll
+                    for (int k = 0; k < kBatch; ++k) tmem_ld8(ta + uint32_t((cq * kChunks + k0 + k) * 8), v[k]);
                     tmem_wait_ld();
-                    uint32_t pk[4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float x0 = mma_ok ? v[2 * i] + sbias[g * kPC + c8 + 2 * i] : 0.f;
-                        const float x1 = mma_ok ? v[2 * i + 1] + sbias[g * kPC + c8 + 2 * i + 1] : 0.f;
-                        pk[i] = uint32_t(bf16_bits_rn(x0)) | (uint32_t(bf16_bits_rn(x1)) << 16);
+                    for (int k = 0; k < kBatch; ++k) {
+                        const int col = (cq * kChunks + k0 + k) * 8;  // accumulator column = g * kPC + channel
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float x0 = mma_ok ? v[k][2 * i] + sbias[col + 2 * i] : 0.f;
+                            const float x1 = mma_ok ? v[k][2 * i + 1] + sbias[col + 2 * i + 1] : 0.f;
+                            pk[i] = uint32_t(bf16_bits_rn(x0)) | (uint32_t(bf16_bits_rn(x1)) << 16);
+                        }
+                        // lanes 2i and 2i+1 hold timesteps 2i and 2i+1: the even
+                        // lane writes the pairs of channels col..col+3, the
+                        // odd lane those of col+4..col+7
+                        const bool odd = lane & 1;
+                        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, odd ? pk[0] : pk[2], 1);
+                        const uint32_t r1 = __shfl_xor_sync(0xffffffffu, odd ? pk[1] : pk[3], 1);
+                        uint4 q;
+                        if (!odd) {
+                            q = make_uint4(__byte_perm(pk[0], r0, 0x5410), __byte_perm(pk[0], r0, 0x7632),
+                                           __byte_perm(pk[1], r1, 0x5410), __byte_perm(pk[1], r1, 0x7632));
+                        } else {
+                            q = make_uint4(__byte_perm(r0, pk[2], 0x5410), __byte_perm(r0, pk[2], 0x7632),
+                                           __byte_perm(r1, pk[3], 0x5410), __byte_perm(r1, pk[3], 0x7632));
+                        }
+                        *reinterpret_cast<uint4*>(su + (trow >> 1) * LY::su_row + (col + (odd ? 4 : 0)) * 4) = q;
                     }
-                    const uint4 qv = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4*>(su + trow * LY::su_row + (g * kPC + c8) * 2) = qv;
-                    if (l < L && d0 + c8 < D)
-                        *reinterpret_cast<uint4*>(p.u + ((b * L + l) * G + g) * D + d0 + c8) = qv;
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);  // this warp is done with the accumulator
             epi_sync();  // su complete
+
 
             // ---- Newton pass 0 on the tile: row group rg, channel c
             const bool cv = d0 + c < D;
@@ -352,9 +373,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
             for (int g = 0; g < G; ++g) aw[g] = cv ? p.a[g * D + d0 + c] : 0.f;
             // state before step l0 at H^0
             const float hp = (l0 == 0 && p.h0 && cv) ? p.h0[b * D + d0 + c] : 0.f;
-            auto gate = [&](int r, int g) {
-                const uint16_t x = *reinterpret_cast<const uint16_t*>(su + r * LY::su_row + (g * kPC + c) * 2);
-                return __uint_as_float(uint32_t(x) << 16);
+            // gate g of timesteps r, r + 1 (r even) as a pair
+            auto gate2 = [&](int r, int g) {
+                const uint32_t x = *reinterpret_cast<const uint32_t*>(su + (r >> 1) * LY::su_row + (g * kPC + c) * 4);
+                return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
             };
             float Jm[kRows], Ov[kRows];  // the step maps, kept for the second sweep
             float r0max = 0.f;
@@ -368,8 +390,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 float2 ua[G], ub[G], fa, fb;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    ua[g] = make_float2(gate(r0 + i, g), gate(r0 + i + 1, g));
-                    ub[g] = make_float2(gate(r0 + i + 2, g), gate(r0 + i + 3, g));
+                    ua[g] = gate2(r0 + i, g);
+                    ub[g] = gate2(r0 + i + 2, g);
                 }
                 Aff2<1> ja, jb;
                 Cell::Packed::Rows2::eval(&sa, ua, &sb, ub, aw2, &fa, &fb, ja, jb);
@@ -391,8 +413,29 @@ __global__ void __launch_bounds__(kPThreads, 1)
             epi_sync();
 
             // epilogue warp 0: the tile's map per channel (two a lane), the
-            // decoupled look-back along the sequence, the carry
-            if (e == 0) {
+            // decoupled look-back along the sequence, the carry.  Meanwhile
+            // the other warps write u to global memory from su: a thread
+            // takes 8 channels of one gate for a pair of timesteps and writes
+            // 16 bytes to each; a row of one gate is 128 contiguous bytes,
+            // written by 8 consecutive threads (whole lines).
+            if (e != 0) {
+                constexpr int kSeg = G * kPC / 8;  // 8-channel pieces of a pair of timesteps
+                for (int j = et - 32; j < (kPM / 2) * kSeg; j += 32 * (kPEpiWarps - 1)) {
+                    const int rp = j / kSeg, q = j - rp * kSeg;
+                    const int g = q / (kPC / 8), c8 = (q - g * (kPC / 8)) * 8;
+                    const uint4* src = reinterpret_cast<const uint4*>(su + rp * LY::su_row + (g * kPC + c8) * 4);
+                    const uint4 w0 = src[0], w1 = src[1];
+                    const uint4 ev = make_uint4(__byte_perm(w0.x, w0.y, 0x5410), __byte_perm(w0.z, w0.w, 0x5410),
+                                                __byte_perm(w1.x, w1.y, 0x5410), __byte_perm(w1.z, w1.w, 0x5410));
+                    const uint4 od = make_uint4(__byte_perm(w0.x, w0.y, 0x7632), __byte_perm(w0.z, w0.w, 0x7632),
+                                                __byte_perm(w1.x, w1.y, 0x7632), __byte_perm(w1.z, w1.w, 0x7632));
+                    const long long l = l0 + 2 * rp;
+                    if (d0 + c8 < D) {
+                        if (l < L) *reinterpret_cast<uint4*>(p.u + ((b * L + l) * G + g) * D + d0 + c8) = ev;
+                        if (l + 1 < L) *reinterpret_cast<uint4*>(p.u + ((b * L + l + 1) * G + g) * D + d0 + c8) = od;
+                    }
+                }
+            } else {
                 const unsigned t_agg = 1u, t_incl = 2u;
                 Map ta[2];
                 float carry[2];
@@ -479,8 +522,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     float2 ua[G], ub[G], fa, fb;
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        ua[g] = make_float2(gate(r0 + i, g), gate(r0 + i + 1, g));
-                        ub[g] = make_float2(gate(r0 + i + 2, g), gate(r0 + i + 3, g));
+                        ua[g] = gate2(r0 + i, g);
+                        ub[g] = gate2(r0 + i + 2, g);
                     }
                     Cell::Packed::Rows2::value(&sa, ua, &sb, ub, aw2, &fa, &fb);
                     const float fv[4] = {fa.x, fa.y, fb.x, fb.y};
