@@ -514,7 +514,7 @@ long long segment_record_floats(int cell, long long BD)
 size_t segment_fold_ws_bytes(int cell, long long B, long long L, long long D)
 {
     if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
-    const long long nf = (L - 1 + kFoldSteps - 1) / kFoldSteps;
+    const long long steps = fold_steps(L), nf = (L - 1 + steps - 1) / steps;
     return align256(size_t(std::max(nf, 1ll)) * (cell == 0 ? 2 : 6) * B * D * 4);
 }
 
@@ -526,11 +526,12 @@ pararnn_status launch_fold(const UT* u, const float* a, const float* s_in, float
     const long long BD = B * D;
     unsigned* res = reinterpret_cast<unsigned*>(rec + R::F * BD);
     CUDA_TRY(cudaMemsetAsync(res, 0, 16, stream));
-    const int nf = int((L - 1 + kFoldSteps - 1) / kFoldSteps);
+    const long long steps = fold_steps(L);
+    const int nf = int((L - 1 + steps - 1) / steps);
     if (nf > 0) {
         const long long threads = B * (D / 4);
         const dim3 grid(unsigned((threads + 127) / 128), unsigned(nf)), block(128);
-        segment_fold_kernel<Cell, UT><<<grid, block, 0, stream>>>(u, a, s_in, part, res, B, L, D);
+        segment_fold_kernel<Cell, UT><<<grid, block, 0, stream>>>(u, a, s_in, part, res, B, L, D, int(steps));
         CUDA_TRY(cudaGetLastError());
         g_launches.fetch_add(1, std::memory_order_relaxed);
     }

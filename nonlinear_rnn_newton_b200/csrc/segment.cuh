@@ -80,10 +80,19 @@ struct SegRecord {
     static __host__ __device__ long long floats(long long BD) { return F * BD + 4; }
 };
 
-// Steps folded per thread in segment_fold_kernel.
-constexpr int kFoldSteps = 128;
+// Steps folded per thread in segment_fold_kernel: the fewest of 64, 128,
+// 256, ... that leave at most kFoldParts parts to compose in order (so that
+// short segments still give every SM several warps, and the parts of a long
+// one stay few for segment_record_kernel's serial composition).
+constexpr int kFoldParts = 256;
+__host__ __device__ inline long long fold_steps(long long Ls)
+{
+    long long steps = 64;
+    while ((Ls - 1 + steps - 1) / steps > kFoldParts) steps *= 2;
+    return steps;
+}
 
-// Fold of steps [1 + f*kFoldSteps, 1 + (f+1)*kFoldSteps) of a segment (f =
+// Fold of steps [1 + f*steps, 1 + (f+1)*steps) of a segment (f =
 // blockIdx.y) for 4 channels a thread: the step maps at H^k (s_in, NULL = the
 // zero guess) composed in order into part [nf][NC][B][D], and max |F| of the
 // steps into *res.  Page: "A sacada: método de Newton" (the Newton step is the
@@ -91,7 +100,8 @@ constexpr int kFoldSteps = 128;
 template <class Cell, class UT>
 __global__ void __launch_bounds__(128) segment_fold_kernel(const UT* __restrict__ u, const float* __restrict__ a,
                                                            const float* __restrict__ s_in, float* __restrict__ part,
-                                                           unsigned* res, long long B, long long Ls, long long D)
+                                                           unsigned* res, long long B, long long Ls, long long D,
+                                                           int steps)
 {
     using Map = typename Cell::Map;
     constexpr int G = Cell::G, NS = Cell::NS, NC = Map::kFloats;
@@ -100,8 +110,8 @@ __global__ void __launch_bounds__(128) segment_fold_kernel(const UT* __restrict_
     float rmax = 0.f;
     if (i < B * D4) {
         const long long b = i / D4, d = (i - b * D4) << 2;
-        const long long l0 = 1 + (long long)blockIdx.y * kFoldSteps;
-        const long long l1 = l0 + kFoldSteps < Ls ? l0 + kFoldSteps : Ls;
+        const long long l0 = 1 + (long long)blockIdx.y * steps;
+        const long long l1 = l0 + steps < Ls ? l0 + steps : Ls;
         float av[G][kV];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -183,6 +193,9 @@ __global__ void __launch_bounds__(256) segment_record_kernel(const UT* __restric
     if (i >= BD) return;
     const long long b = i / D, d = i - b * D;
     Map acc = Map::identity();
+    // (unrolled, so that the reads of several parts are in flight while the
+    // compositions form the chain)
+#pragma unroll 8
     for (int f = 0; f < nf; ++f) {
         Map m;
 #pragma unroll

@@ -135,10 +135,13 @@ def test_segment_checks(capi):
     assert lib.pararnn_segment_record_floats(1, 2, 16) == (2 + 2 + 3) * 32 + 4
     assert lib.pararnn_segment_record_floats(2, 2, 16) == (6 + 4 + 4) * 32 + 4
     assert lib.pararnn_segment_record_floats(3, 2, 16) == 0
-    # partial folds of 128 steps: steps 2..L of the segment
+    # partial folds of steps 2..L of the segment, 64 steps each, or twice as
+    # many steps until at most 256 parts remain
     assert lib.pararnn_segment_fold_workspace_size(1, 1, 129, 16) == 256
-    assert lib.pararnn_segment_fold_workspace_size(2, 4, 257, 64) == 2 * 6 * 4 * 64 * 4
-    assert lib.pararnn_segment_fold_workspace_size(2, 4, 258, 64) == 3 * 6 * 4 * 64 * 4
+    assert lib.pararnn_segment_fold_workspace_size(2, 4, 257, 64) == 4 * 6 * 4 * 64 * 4
+    assert lib.pararnn_segment_fold_workspace_size(2, 4, 258, 64) == 5 * 6 * 4 * 64 * 4
+    assert lib.pararnn_segment_fold_workspace_size(1, 1, 64 * 256 + 1, 16) == 256 * 2 * 16 * 4
+    assert lib.pararnn_segment_fold_workspace_size(1, 1, 64 * 256 + 2, 16) == (129 * 2 * 16 * 4 + 255) // 256 * 256
 
 
 def test_decode_step_checks(capi):

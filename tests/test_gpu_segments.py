@@ -82,7 +82,7 @@ def test_segment_stopping_rules(cuda):
 
 def test_segment_memory_is_the_iterate_plus_small_buffers(cuda):
     """A segment holds its iterate (updated in place), B*D-sized buffers, the
-    fold's partial maps (one per 128 steps) and the fused pass's workspace:
+    fold's partial maps (one per 64 steps or more) and the fused pass's workspace:
     nothing else of the iterate's size."""
     B, Ls, D = 2, 1024, 256
     u = torch.zeros((B, Ls, 3, D), dtype=torch.bfloat16, device=cuda)
