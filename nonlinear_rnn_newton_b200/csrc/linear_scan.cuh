@@ -85,7 +85,7 @@ __device__ __forceinline__ void linear_gru_maps2(float2 uza, float2 uca, float2 
 // LB: look-backs step back over aggregates (1), wait for inclusive values (0)
 // or follow p.lb_walk (2).
 template <class UT, int CW, int R, int LB = 2>
-__global__ void __launch_bounds__(32 * (CW + 1), CW < 8 ? 2 : 1)
+__global__ void __launch_bounds__(32 * (CW + 1), 1)
     linear_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const LinScanParams p)
 {
     using LY = LinScanLayout<UT, CW, R>;
