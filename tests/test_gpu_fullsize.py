@@ -37,6 +37,24 @@ def test_gru_fullsize_sampled(cuda, w):
     del xd, h
 
 
+@pytest.mark.parametrize("w", [W.GRU, W.GRU_SWEEP[4]], ids=lambda w: w.name)
+def test_linear_scan_fullsize_sampled(cuda, w):
+    """The plain linear scan (the zero-weight GRU) on the bench's inputs and
+    launch: sampled channels against the oracle's stepping with a = 0."""
+    x = W.make_inputs(w, seed=0)
+    xd = x.to(cuda)
+    h = P().pararnn_linear_scan(xd.u, xd.h0)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(h).all())
+    x0 = W.Inputs(u=x.u, a=torch.zeros_like(x.a), h0=x.h0)
+    picks = H.sample_channels(w.B, w.D, 24)
+    ref = H.gru_seq_channels(x0, picks)
+    hc = h.cpu()
+    for (b, d), v in ref.items():
+        assert H.max_abs(hc[b, :, d].double().numpy(), v) <= TOL_STATE, (b, d)
+    del xd, h
+
+
 def test_lstm_fullsize_sampled(cuda):
     w = W.LSTM
     x = W.make_inputs(w, seed=0)
