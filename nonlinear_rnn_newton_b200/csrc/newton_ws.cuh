@@ -322,6 +322,10 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     prefix(wb, run);
                 }
                 float y[NS][kV];
+                // waiting for inclusive values needs none of this group's
+                // maps: a group's first carry then goes out before the second
+                // tile's folds are composed
+                const bool early = !walk && !local;
                 if (local) {
                     // carry = inclusive value of the group's previous tile
 #pragma unroll
@@ -330,6 +334,25 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                         for (int j = 0; j < kV; ++j) y[q][j] = y_inc[q][j];
                     pre_done = false;
                 } else {
+                    if (early) {
+                        if (c > 0) {
+                            ok = lookback_resolve<Map, NS, false>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) &&
+                                 ok;
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) {
+                                F4 x{{0.f, 0.f, 0.f, 0.f}};
+                                if (dch < D && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+#pragma unroll
+                                for (int j = 0; j < kV; ++j) y[q][j] = x.v[j];
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) store4(car + q * kDc + lane * kV, y[q]);
+                        if (!__all_sync(0xffffffffu, ok) && lane == 0) s_int[0] = 1;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar_carry[wb]);
+                    }
                     // the group's second tile (the next in the ring): its
                     // prefixes now, while the look-back read is in flight
                     bool two = false;
@@ -348,27 +371,25 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             ok = false;  // the group's tiles are always issued back to back
                         }
                     }
-                    if (c > 0) {
-                        // the group's aggregate (both tiles' maps composed)
-                        // goes out first, for look-backs that step over it
-                        if (walk) {
+                    if (!early) {
+                        if (c > 0) {
+                            // stepping back: the group's aggregate (both
+                            // tiles' maps composed) goes out first, for
+                            // look-backs that step over it
                             Map gagg[kV];
 #pragma unroll
                             for (int j = 0; j < kV; ++j) gagg[j] = two ? compose(run_pre[j], run[j]) : run[j];
                             publish_aggregate<Map, NS>(p.desc, gt, k, gagg, lane);
                             ok = lookback_resolve<Map, NS, true>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) && ok;
                         } else {
-                            ok = lookback_resolve<Map, NS, false>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) &&
-                                 ok;
-                        }
-                    } else {
-                        // the sequence's first group: the initial state
+                            // the sequence's first group: the initial state
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) {
-                            F4 x{{0.f, 0.f, 0.f, 0.f}};
-                            if (dch < D && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
+                            for (int q = 0; q < NS; ++q) {
+                                F4 x{{0.f, 0.f, 0.f, 0.f}};
+                                if (dch < D && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
 #pragma unroll
-                            for (int j = 0; j < kV; ++j) y[q][j] = x.v[j];
+                                for (int j = 0; j < kV; ++j) y[q][j] = x.v[j];
+                            }
                         }
                     }
                 }
@@ -396,11 +417,13 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     }
                     publish_inclusive<Map, NS>(p.desc, gt, k, incl, lane);
                 }
+                if (!early) {
 #pragma unroll
-                for (int q = 0; q < NS; ++q) store4(car + q * kDc + lane * kV, y[q]);
+                    for (int q = 0; q < NS; ++q) store4(car + q * kDc + lane * kV, y[q]);
+                }
                 if (!__all_sync(0xffffffffu, ok) && lane == 0) s_int[0] = 1;
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar_carry[wb]);
+                if (!early && lane == 0) mbar_arrive(&bar_carry[wb]);
                 // refill the stage released by the tile before this one
                 if (n >= 1) {
                     const int sp = (n - 1) % kStages;
