@@ -715,7 +715,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="only the headline workload (the other solve "
                     "workloads run by default on one GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=-1,
+                    help="steps of the end-to-end run (-1: as many as --steps; 0: none)")
     ap.add_argument("--baselines", type=int, default=1, help="also time the sequential GPU kernel and "
                     "the plain linear scan on the headline's input (GRU workloads)")
     ap.add_argument("--decode", action="store_true", help="add the decode-step timings (CUDA graph of steps)")
@@ -796,12 +797,13 @@ def main():
                    "traffic": profile_traffic("adjoint_kernel", w.name)}
 
     e2e = None
-    if args.e2e_steps > 0:
+    e2e_steps = args.steps if args.e2e_steps < 0 else args.e2e_steps
+    if e2e_steps > 0:
         barrier(world)
-        ems, h2d, d2h = run_e2e(w, x, dev, args.e2e_steps)
+        ems, h2d, d2h = run_e2e(w, x, dev, e2e_steps)
         ems = max_over_ranks(ems, world)
         e2e = {"value": job_value(w.N, world, ems), "unit": UNIT, "ms_per_step": ems,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     baselines = None
     if args.baselines and w.cell == "gru":
