@@ -56,6 +56,31 @@ def test_segments_match_single_gpu_and_oracle(cuda, cell, lens, dt):
     assert H.max_abs(Hs.cpu(), seq) <= 1e-4
 
 
+def test_long_segments_fold_longer_parts(cuda):
+    """Segments longer than 64 * 256 steps fold 128 steps a part (and a short
+    one 64): the split solve still matches the single-GPU solve and sampled
+    oracle channels."""
+    lens = [20000, 700]
+    B, L, D = 1, sum(lens), 64
+    w = W.custom("gru", B, L, D, "bf16", h0_std=0.1)
+    x = W.make_inputs(w, seed=21)
+    xd = x.to(cuda)
+    s0 = xd.h0[None].contiguous()
+    edges = np.cumsum([0] + lens)
+    segs = [SH.Segment("gru", xd.u[:, edges[r]:edges[r + 1]].contiguous(), xd.a, r) for r in range(len(lens))]
+    it, res, st = SH.solve_segments(segs, SH.LocalComm(), s0, w.tol, w.max_iters)
+    Hs = torch.cat([sg.H for sg in segs], dim=2)[0]
+    h, it1, r1, st1 = P().pararnn_gru_solve(xd.u, xd.a, xd.h0)
+    torch.cuda.synchronize()
+    assert st == 0 and st1 == 0 and abs(it - it1) <= 1, (it, it1)
+    assert float((Hs - h).abs().max()) <= 1e-5
+    picks = H.sample_channels(B, D, 6)
+    ref = H.gru_seq_channels(x, picks)
+    hc = Hs.cpu()
+    for (b, d), v in ref.items():
+        assert H.max_abs(hc[b, :, d].double().numpy(), v) <= 1e-4, (b, d)
+
+
 def test_segment_stopping_rules(cuda):
     """max_iters = 0 and a huge tol stop at the zero guess; max_iters = 1
     gives the oracle's first iterate; each piece checks its arguments."""
