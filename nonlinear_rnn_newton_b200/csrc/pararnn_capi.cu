@@ -56,9 +56,6 @@ pararnn_status fail(pararnn_status s, const char* fmt, ...)
         if (s_ != PARARNN_OK) return s_;          \
     } while (0)
 
-#ifndef PARARNN_ADJ_ROWS
-#define PARARNN_ADJ_ROWS 4
-#endif
 constexpr size_t kSelftestWorkspace = 16384;
 #ifndef PARARNN_WS_GRU_WARPS
 #define PARARNN_WS_GRU_WARPS 15
@@ -75,7 +72,6 @@ template <class UT> constexpr int lstm_lc() { return 2 * lstm_tile_arg<UT>(); }
 // workspace sizing uses the shortest tile (most tiles) of either input dtype
 constexpr int kLcGru = gru_lc<float>() < gru_lc<uint16_t>() ? gru_lc<float>() : gru_lc<uint16_t>();
 constexpr int kLcLstm = lstm_lc<float>() < lstm_lc<uint16_t>() ? lstm_lc<float>() : lstm_lc<uint16_t>();
-constexpr int kLcAdj = kWarps * PARARNN_ADJ_ROWS;    // adjoints
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -821,7 +817,7 @@ pararnn_status adjoint_async(int cell, const void* u, pararnn_dtype dt, const fl
         TRY(check_ptr(dc0, "dc0", false));
     }
     Shape s;
-    TRY(make_shape(B, L, D, kLcAdj, &s));
+    TRY(make_shape(B, L, D, cell == 0 ? adj_lc_min<GruCell>() : adj_lc_min<LstmCell>(), &s));
     TRY(check_workspace(ws, ws_bytes, adjoint_ws_bytes(cell, B, L, D)));
     if (cell == 0) {
         const float* s0[2] = {h0, nullptr};
