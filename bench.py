@@ -98,7 +98,7 @@ def adjoint_bytes(w: W.Workload) -> int:
 _COMMON = ["device_common.cuh", "pararnn_internal.h", "cells.cuh", "scan_common.cuh"]
 KERNEL_SOURCES = {
     "newton_solve_ws_kernel": _COMMON + ["newton.cuh", "newton_ws.cuh"],
-    "adjoint_kernel": _COMMON + ["adjoint.cuh", "adjoint_ws.cuh"],
+    "adjoint_ws_kernel": _COMMON + ["adjoint.cuh", "adjoint_ws.cuh"],
     "project_pass0_kernel": _COMMON + ["project.cuh"],
 }
 
@@ -344,9 +344,9 @@ def measure(w, dev, stream, reps=10, warmup=3, baselines=True):
     if w.train:
         adj_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
         ab = adjoint_bytes(w)
-        out["adjoint"] = {"kernel": "adjoint_kernel", "kernel_ms_mean": adj_ms, "algorithmic_bytes_per_launch": ab,
+        out["adjoint"] = {"kernel": "adjoint_ws_kernel", "kernel_ms_mean": adj_ms, "algorithmic_bytes_per_launch": ab,
                           "achieved": ab / (adj_ms * 1e-3) / 1e9, "frac": ab / (adj_ms * 1e-3) / 1e9 / peak,
-                          "traffic": profile_traffic("adjoint_kernel", w.name)}
+                          "traffic": profile_traffic("adjoint_ws_kernel", w.name)}
     if baselines and w.cell == "gru":
         out["baselines"] = time_baselines(w, xd, st.out[0], stream, dev)
     del st, xd
@@ -794,7 +794,7 @@ def main():
         ab = adjoint_bytes(w)
         adjoint = {"kernel_ms_mean": adj_ms, "algorithmic_bytes_per_launch": ab,
                    "achieved": ab / (adj_ms * 1e-3) / 1e9, "frac": ab / (adj_ms * 1e-3) / 1e9 / peak,
-                   "traffic": profile_traffic("adjoint_kernel", w.name)}
+                   "traffic": profile_traffic("adjoint_ws_kernel", w.name)}
 
     e2e = None
     e2e_steps = args.steps if args.e2e_steps < 0 else args.e2e_steps

@@ -18,8 +18,7 @@
 // gradient of the initial state is mu_1.
 //
 // This header holds what the scan kernel shares with the host: its
-// parameter block, the fixed-order reduction of da, and the self tests of
-// the bounded waits.
+// parameter block and the fixed-order reduction of da.
 #pragma once
 
 #include <climits>
@@ -70,29 +69,6 @@ __global__ void __launch_bounds__(256) da_reduce_kernel(const float* __restrict_
         for (int i = 0; i < 8; ++i) t += red[i][threadIdx.x];
         da[col] = t;
     }
-}
-
-// ------------------------------------------------------------ self tests
-// Each runs one of the bounded waits against a condition nothing satisfies.
-
-// The look-back of tile 1 whose predecessor (tile 0) never publishes.
-__global__ void selftest_lookback_kernel(unsigned long long* desc, int* err, unsigned long long limit_ns)
-{
-    Aff<1> ta[kV];
-    float init[1][kV], carry[1][kV];
-#pragma unroll
-    for (int j = 0; j < kV; ++j) {
-        ta[j] = Aff<1>::identity();
-        init[0][j] = 0.f;
-    }
-    (void)lookback<Aff<1>, 1>(1, 1, true, 0, ta, init, carry, desc, threadIdx.x & 31, err, limit_ns);
-}
-
-__global__ void selftest_barrier_kernel(unsigned* counter, int* err, unsigned long long limit_ns)
-{
-    __shared__ int s_flag;
-    if (blockIdx.x == gridDim.x - 1) return;  // this CTA never arrives
-    (void)grid_barrier(counter, 0u, err, limit_ns, &s_flag);
 }
 
 }  // namespace pararnn

@@ -156,21 +156,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* tm, in
         : "memory");
 }
 
-// Tiled prefetch into L2 only (no shared memory, no completion tracking).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* tm, int c0, int c1, int c2)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tm), "r"(c0),
-                 "r"(c1), "r"(c2)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* tm, int c0, int c1, int c2, int c3)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(tm), "r"(c0),
-                 "r"(c1), "r"(c2), "r"(c3)
-                 : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tm) : "memory");
@@ -326,25 +311,9 @@ __device__ __forceinline__ void stcgv(float* p, const float* v)
     else __stcg(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
 }
 
-__device__ __forceinline__ F4 ldcg4(const float* p)
-{
-    float4 w = __ldcg(reinterpret_cast<const float4*>(p));
-    F4 r;
-    r.v[0] = w.x;
-    r.v[1] = w.y;
-    r.v[2] = w.z;
-    r.v[3] = w.w;
-    return r;
-}
-
 __device__ __forceinline__ void store4(float* p, const float* v)
 {
     *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-}
-
-__device__ __forceinline__ void stcg4(float* p, const float* v)
-{
-    __stcg(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
 }
 
 // --------------------------------------------------------- elementary math
@@ -424,19 +393,6 @@ __device__ __forceinline__ void sigmoid_tanh(float x, float y, float& sx, float&
 __device__ __forceinline__ float tanh_fast(float x)
 {
     return fmaf(-2.0f, rcp_approx(1.0f + ex2_approx(2.0f * kLog2e * x)), 1.0f);
-}
-
-__device__ __forceinline__ float sigmoid_fast(float x)
-{
-    return rcp_approx(1.0f + ex2_approx(-kLog2e * x));
-}
-
-// |x| as ordered bits: for non-negative floats the unsigned bit patterns
-// order like the values, and any NaN orders above +inf, so an unsigned max
-// over these keeps NaN and inf visible (unlike fmaxf, which drops NaN).
-__device__ __forceinline__ unsigned abs_bits(float x)
-{
-    return __float_as_uint(x) & 0x7fffffffu;
 }
 
 }  // namespace pararnn

@@ -23,6 +23,7 @@
 #include "decode.cuh"
 #include "segment.cuh"
 #include "adjoint.cuh"
+#include "selftest.cuh"
 #include "adjoint_ws.cuh"
 #include "linear_scan.cuh"
 #include "project.cuh"
@@ -261,7 +262,7 @@ pararnn_status device_info(int* sms)
 }
 
 template <class K>
-pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid, int threads = kThreads)
+pararnn_status resident_grid(K kern, size_t smem, int n_tiles, int* grid, int threads)
 {
     int sms = 0;
     TRY(device_info(&sms));

@@ -9,15 +9,6 @@
 
 namespace pararnn {
 
-#ifndef PARARNN_WARPS
-#define PARARNN_WARPS 8
-#endif
-constexpr int kWarps = PARARNN_WARPS;  // warps per CTA: each owns T consecutive timesteps
-constexpr int kThreads = 32 * kWarps;  // threads per CTA
-#ifndef PARARNN_MINB
-#define PARARNN_MINB (16 / PARARNN_WARPS)
-#endif
-constexpr int kMinBlocks = PARARNN_MINB;  // CTAs per SM the kernels are register-budgeted for
 constexpr int kV = 4;              // channels per lane
 constexpr int kDc = 32 * kV;       // channels per tile (one per lane x kV)
 

@@ -1,5 +1,6 @@
-// Chunked parallel scan of affine maps, shared by the Newton solve, the
-// adjoint and the linear-scan baseline.
+// The parts of the chunked parallel scan of affine maps that the Newton
+// solve, the adjoint and the linear-scan baseline share: the tagged words
+// through which tiles hand values to one another, and the look-back.
 //
 // Page: "ParaRNN: Apple destrava treino paralelo de RNNs não-lineares e escala
 // pra 7B parâmetros", section "O compromisso que SSMs fizeram": a linear
@@ -7,96 +8,19 @@
 // (O(log L) depth) instead of step by step; section "A sacada: método de
 // Newton": every Newton iteration is such a linear recurrence.
 //
-// Three levels: (1) each thread folds its T timesteps serially in registers;
-// (2) a warp-shuffle scan combines the warps' segments of a tile, each
-// channel group handled by kWarps lanes; (3) a decoupled look-back combines tiles
-// across CTAs: every tile publishes its aggregate right away, then walks back
-// over predecessors' aggregates until it meets an inclusive prefix, and
-// publishes its own inclusive value.  Values travel as tagged 64-bit words
-// (each word is its own ready flag, so no fences); every wait is bounded.
+// Every scan kernel works in three levels: (1) each compute warp folds the
+// maps of its two steps of a tile in registers; (2) the CTA's control warp
+// composes the warps' folds into exclusive prefixes; (3) tiles (or groups of
+// tiles) are chained across CTAs: each publishes its aggregate, resolves the
+// value entering it from its predecessors' published words (stepping back
+// over aggregates, or waiting for the predecessor's inclusive value), and
+// publishes its inclusive value.  Values travel as tagged 64-bit words (each
+// word is its own ready flag, so no fences); every wait is bounded.
 #pragma once
 
 #include "cells.cuh"
 
 namespace pararnn {
-
-constexpr int kScanPad = kDc + 4;  // padded scratch row (floats): conflict-free strided reads
-
-template <class Map>
-__device__ __forceinline__ Map shfl_up_map8(const Map& x, int delta)
-{
-    Map r;
-#pragma unroll
-    for (int i = 0; i < Map::kFloats; ++i) r.set(i, __shfl_up_sync(0xffffffffu, x.get(i), delta, kWarps));
-    return r;
-}
-
-// Write a thread's kV per-channel maps to segment position `pos` of the scratch
-// [NC][kWarps][kScanPad].
-template <class Map>
-__device__ __forceinline__ void scan_put(float* scan, int pos, int lane, const Map (&m)[kV])
-{
-#pragma unroll
-    for (int i = 0; i < Map::kFloats; ++i) {
-        float v4[kV];
-#pragma unroll
-        for (int j = 0; j < kV; ++j) v4[j] = m[j].get(i);
-        store4(scan + (i * kWarps + pos) * kScanPad + lane * kV, v4);
-    }
-}
-
-// Read one channel's map at segment position `pos`.
-template <class Map>
-__device__ __forceinline__ Map scan_get(const float* scan, int pos, int ch)
-{
-    Map m;
-#pragma unroll
-    for (int i = 0; i < Map::kFloats; ++i) m.set(i, scan[(i * kWarps + pos) * kScanPad + ch]);
-    return m;
-}
-
-// In-place exclusive scan over the kWarps segment positions of the scratch,
-// for all kDc channels; the full-tile aggregate goes to tagg [NC][kDc].
-// Called by all kThreads threads between two __syncthreads.
-template <class Map>
-__device__ __forceinline__ void cta_segment_scan(float* scan, float* tagg, int tid)
-{
-    constexpr int NC = Map::kFloats;
-    const int grp = tid / kWarps;  // channels grp*kV .. grp*kV+kV-1
-    const int seg = tid % kWarps;  // segment position
-    Map x[kV];
-#pragma unroll
-    for (int i = 0; i < NC; ++i) {
-        F4 v = load4(scan + (i * kWarps + seg) * kScanPad + grp * kV);
-#pragma unroll
-        for (int j = 0; j < kV; ++j) x[j].set(i, v.v[j]);
-    }
-#pragma unroll
-    for (int off = 1; off < kWarps; off <<= 1) {
-#pragma unroll
-        for (int j = 0; j < kV; ++j) {
-            Map y = shfl_up_map8(x[j], off);
-            if (seg >= off) x[j] = compose(x[j], y);
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < kV; ++j) {
-        Map y = shfl_up_map8(x[j], 1);
-        if (seg == 0) y = Map::identity();
-        if (seg == kWarps - 1) {
-#pragma unroll
-            for (int i = 0; i < NC; ++i) tagg[i * kDc + grp * kV + j] = x[j].get(i);
-        }
-        x[j] = y;
-    }
-#pragma unroll
-    for (int i = 0; i < NC; ++i) {
-        float v4[kV];
-#pragma unroll
-        for (int j = 0; j < kV; ++j) v4[j] = x[j].get(i);
-        store4(scan + (i * kWarps + seg) * kScanPad + grp * kV, v4);
-    }
-}
 
 // Published values are tagged 64-bit words: the float in the low half, a tag
 // in the high half.  An aligned 64-bit access is single-copy atomic, so a
@@ -160,7 +84,7 @@ __device__ __forceinline__ bool unpack_words(const unsigned long long (&w)[N], f
 
 // First look-back probe: the words of the predecessor tile (its inclusive
 // value and its aggregate), loaded early so that the round trip overlaps
-// whatever the caller does before calling lookback().
+// whatever the caller does before calling lookback_resolve().
 template <class Map, int NS>
 struct LookbackProbe {
     unsigned long long wi[kV * NS];
@@ -288,54 +212,6 @@ __device__ __forceinline__ bool lookback_resolve(int ticket, int stride, int epo
         }
     }
     return __all_sync(0xffffffffu, ok);
-}
-
-// Decoupled look-back of one tile with aggregate `ta`: publishes the
-// aggregate (if there is a predecessor), resolves the carry (`init` for the
-// first tile of a sequence) and publishes the inclusive value
-// apply(ta, carry).  False if a wait gave up.
-template <class Map, int NS>
-__device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, int epoch, const Map (&ta)[kV],
-                                         const float (&init)[NS][kV], float (&carry)[NS][kV],
-                                         unsigned long long* desc, int lane, int* err,
-                                         unsigned long long wait_ns, LookbackProbe<Map, NS>& pr)
-{
-    bool ok = true;
-    if (has_pred) {
-        publish_aggregate<Map, NS>(desc, ticket, epoch, ta, lane);
-        ok = lookback_resolve<Map, NS, true>(ticket, stride, epoch, carry, desc, lane, err, wait_ns, pr);
-    } else {
-#pragma unroll
-        for (int q = 0; q < NS; ++q)
-#pragma unroll
-            for (int j = 0; j < kV; ++j) carry[q][j] = init[q][j];
-    }
-    if (ok) {
-        float incl[NS][kV];
-#pragma unroll
-        for (int j = 0; j < kV; ++j) {
-            float x[NS], y[NS];
-#pragma unroll
-            for (int q = 0; q < NS; ++q) x[q] = carry[q][j];
-            apply(ta[j], x, y);
-#pragma unroll
-            for (int q = 0; q < NS; ++q) incl[q][j] = y[q];
-        }
-        publish_inclusive<Map, NS>(desc, ticket, epoch, incl, lane);
-    }
-    return ok;
-}
-
-// Look-back without an early probe.
-template <class Map, int NS>
-__device__ __forceinline__ bool lookback(int ticket, int stride, bool has_pred, int epoch, const Map (&ta)[kV],
-                                         const float (&init)[NS][kV], float (&carry)[NS][kV],
-                                         unsigned long long* desc, int lane, int* err,
-                                         unsigned long long wait_ns)
-{
-    LookbackProbe<Map, NS> pr;
-    if (has_pred) lookback_probe(pr, ticket - stride, desc, lane);
-    return lookback<Map, NS>(ticket, stride, has_pred, epoch, ta, init, carry, desc, lane, err, wait_ns, pr);
 }
 
 }  // namespace pararnn
