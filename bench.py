@@ -17,9 +17,9 @@ on the data path) and the time is the max over ranks.
 On one GPU the same line also carries, under "configs", every other solve
 workload (ParaGRU and ParaLSTM at B=8, L=4096, D=1024; the B=1, D=2048
 sequence-length sweep with the sequential GPU kernel and the plain linear scan
-at each L; the ParaLSTM training step, solve plus adjoint, at B=4, L=16384,
-D=2048), each with its roofline and per-pass figures, and the CPU oracle's
-sequential stepping timed on all host cores and on one core.
+at each L; the ParaLSTM and ParaGRU training steps, solve plus adjoint, at
+B=4, L=16384, D=2048), each with its roofline and per-pass figures, and the
+CPU oracle's sequential stepping timed on all host cores and on one core.
 
 Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle on a
 bounded sample of the same workload instead (the reference arm; rank 0 only).
@@ -413,7 +413,7 @@ def run_configs(headline, dev, stream):
     """Every solve workload except the headline, one after another, and the
     solve from the layer input (the fused input projection)."""
     out = {}
-    for w in (W.GRU, W.LSTM) + W.GRU_SWEEP + (W.LSTM_TRAIN,):
+    for w in (W.GRU, W.LSTM) + W.GRU_SWEEP + (W.LSTM_TRAIN, W.GRU_TRAIN):
         if w.name == headline.name:
             continue
         out[w.name] = measure(w, dev, stream)

@@ -60,7 +60,8 @@ struct AdjointWsLayout {
     static constexpr size_t misc_bytes = a128((2 * kStages + 2 * kWork) * 8 + kStages * 16 + 8 * 4);
     static constexpr size_t smem_bytes = off_misc + misc_bytes;
     static constexpr int threads = 32 * (CW + 1);
-    static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
+    // descriptors hold inclusive values only: every look-back waits for them
+    static constexpr int desc_words = TileDesc<typename Cell::Map, NS, false>::words;
     static constexpr bool fits = smem_bytes <= 232448;
 };
 
@@ -79,6 +80,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 {
     using LY = AdjointWsLayout<Cell, UT, CW>;
     using Map = typename Cell::Map;
+    using TD = TileDesc<Map, Cell::NS, false>;  // inclusive values only
     constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc;
     constexpr int kStages = LY::kStages, kWork = LY::kWork;
     static_assert(LY::fits, "shared memory");
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 bool ok = mbar_wait_bounded(&bar_aggr[wb], uint32_t(n / kWork) & 1u, err, p.wait_ns);
                 LookbackProbe<Map, NS> pr;
                 const bool has_pred = c < p.n_chunks - 1;  // a later chunk exists
-                if (has_pred) lookback_probe<Map, NS, false>(pr, ticket - BS, p.desc, lane);
+                if (has_pred) lookback_probe<Map, NS, false, TD>(pr, ticket - BS, p.desc, lane);
                 // folds -> exclusive prefixes in place, latest segment first;
                 // their composition is the tile's map
                 float* agg = reinterpret_cast<float*>(work_at(wb) + LY::off_agg);
@@ -197,7 +199,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 #pragma unroll
                     for (int j = 0; j < kV; ++j) y[q][j] = 0.f;
                 if (has_pred)
-                    ok = lookback_resolve<Map, NS, false>(ticket, BS, 0, y, p.desc, lane, err, p.wait_ns, pr) && ok;
+                    ok = lookback_resolve<Map, NS, false, TD>(ticket, BS, 0, y, p.desc, lane, err, p.wait_ns, pr) && ok;
                 if (__all_sync(0xffffffffu, ok)) {
                     float incl[NS][kV];
 #pragma unroll
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 #pragma unroll
                         for (int q = 0; q < NS; ++q) incl[q][j] = z[q];
                     }
-                    publish_inclusive<Map, NS>(p.desc, ticket, 0, incl, lane);
+                    publish_inclusive<Map, NS, TD>(p.desc, ticket, 0, incl, lane);
                 }
                 float* car = reinterpret_cast<float*>(work_at(wb) + LY::off_carry);
 #pragma unroll

@@ -98,7 +98,6 @@ struct NewtonWsLayout {
         a128((2 * kStages + 2 * kWork) * 8 + kStages * 16 + 8 * 4 + 2 * (CWT + 1) * 4);
     static constexpr size_t smem_bytes = off_misc + misc_bytes;
     static constexpr int threads = 32 * (CWT + 1);
-    static constexpr int desc_words = TileDesc<typename Cell::Map, NS>::words;
     static constexpr bool fits = smem_bytes <= 232448;  // opt-in shared memory per CTA
 };
 
@@ -122,6 +121,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
     // look-backs step back over aggregates (LB = 1), wait for inclusive
     // values (LB = 0), or follow p.lb_walk (LB = 2)
     const bool walk = LB == 2 ? p.lb_walk != 0 : LB == 1;
+    // descriptors: inclusive values only when no look-back steps back
+    using TD = TileDesc<Map, NS, LB != 0>;
     static_assert(LY::fits, "shared memory");
 
     extern __shared__ __align__(128) unsigned char smem[];
@@ -316,8 +317,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     // first look-back read, in flight while the folds are composed
                     // (issued only now, so that it sees predecessors as late as possible)
                     if (c > 0 && !local) {
-                        if (walk) lookback_probe<Map, NS, true>(pr, gt - BS, p.desc, lane);
-                        else lookback_probe<Map, NS, false>(pr, gt - BS, p.desc, lane);
+                        if (walk) lookback_probe<Map, NS, LB != 0, TD>(pr, gt - BS, p.desc, lane);
+                        else lookback_probe<Map, NS, false, TD>(pr, gt - BS, p.desc, lane);
                     }
                     prefix(wb, run);
                 }
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 } else {
                     if (early) {
                         if (c > 0) {
-                            ok = lookback_resolve<Map, NS, false>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) &&
+                            ok = lookback_resolve<Map, NS, false, TD>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) &&
                                  ok;
                         } else {
 #pragma unroll
@@ -379,8 +380,12 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             Map gagg[kV];
 #pragma unroll
                             for (int j = 0; j < kV; ++j) gagg[j] = two ? compose(run_pre[j], run[j]) : run[j];
-                            publish_aggregate<Map, NS>(p.desc, gt, k, gagg, lane);
-                            ok = lookback_resolve<Map, NS, true>(gt, BS, k, y, p.desc, lane, err, p.wait_ns, pr) && ok;
+                            if constexpr (LB != 0) {  // (with LB = 0 every head carry goes out early)
+                                publish_aggregate<Map, NS, TD>(p.desc, gt, k, gagg, lane);
+                                ok = lookback_resolve<Map, NS, true, TD>(gt, BS, k, y, p.desc, lane, err, p.wait_ns,
+                                                                         pr) &&
+                                     ok;
+                            }
                         } else {
                             // the sequence's first group: the initial state
 #pragma unroll
@@ -415,7 +420,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
 #pragma unroll
                         for (int q = 0; q < NS; ++q) incl[q][j] = pre_done ? z[q] : x[q];
                     }
-                    publish_inclusive<Map, NS>(p.desc, gt, k, incl, lane);
+                    publish_inclusive<Map, NS, TD>(p.desc, gt, k, incl, lane);
                 }
                 if (!early) {
 #pragma unroll

@@ -294,7 +294,11 @@ pararnn_status launch_newton_k(const Shape& s, const void* u, pararnn_dtype dt, 
     if (s.Lc != KL::Lc) return fail(PARARNN_ERR_INVALID_ARG, "internal: tile rows %d != kernel rows %d", s.Lc, KL::Lc);
     const ScanLayout ly = scan_layout(s, desc_words, solve_bnd_bytes(s, NS), solve_descs(s));
     unsigned char* wsb = static_cast<unsigned char*>(ws);
-    if (zero_ws) CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));  // header + descriptors
+    // header + descriptors; waiting look-backs (LB = 0) use the leading part
+    // of the region only, as descriptors without aggregates
+    const size_t zero_bytes =
+        LB == 0 ? ly.desc + size_t(solve_descs(s)) * TileDesc<typename Cell::Map, NS, false>::words * 8 : ly.extra;
+    if (zero_ws) CUDA_TRY(cudaMemsetAsync(ws, 0, zero_bytes, stream));
 
     CUtensorMap tu, t0, t1;
     TRY(map_gates(&tu, u, dt, Cell::G, Cell::G, s, KL::Lc));
@@ -720,9 +724,15 @@ pararnn_status project_solve_async(const void* x, const void* w, const float* bi
 // Compute warps (two steps each) of the warp-specialised adjoint per cell and
 // gate dtype; fp32 gates need twice the staging space, so their tiles are half
 // as long.
+#ifndef PARARNN_ADJ_GRU_WARPS
+#define PARARNN_ADJ_GRU_WARPS 14
+#endif
+#ifndef PARARNN_ADJ_LSTM_WARPS
+#define PARARNN_ADJ_LSTM_WARPS 7
+#endif
 template <class Cell, class UT> constexpr int adj_warps()
 {
-    return (Cell::NS == 1 ? 11 : 7) / (sizeof(UT) == 2 ? 1 : 2);
+    return (Cell::NS == 1 ? PARARNN_ADJ_GRU_WARPS : PARARNN_ADJ_LSTM_WARPS) / (sizeof(UT) == 2 ? 1 : 2);
 }
 // workspace sizing uses the shortest tile (most tiles) of either gate dtype
 template <class Cell> constexpr int adj_lc_min() { return 2 * adj_warps<Cell, float>(); }
@@ -737,7 +747,7 @@ size_t adjoint_ws_bytes(int cell, long long B, long long L, long long D)
     memcpy(t_err, saved, sizeof(t_err));
     if (st != PARARNN_OK) return 0;
     const int G = cell == 0 ? 3 : 4;
-    const int desc = cell == 0 ? TileDesc<Aff<1>, 1>::words : TileDesc<Aff<2>, 2>::words;
+    const int desc = cell == 0 ? TileDesc<Aff<1>, 1, false>::words : TileDesc<Aff<2>, 2, false>::words;
     return scan_layout(s, desc, size_t(s.n_tiles) * G * kDc * 4).total;
 }
 

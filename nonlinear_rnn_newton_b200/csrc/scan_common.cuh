@@ -43,12 +43,15 @@ __device__ __forceinline__ void ld_words2(const unsigned long long* p, unsigned 
     asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
 
-// Descriptor of one tile in the workspace (tagged words):
-//   aggregates [32 lanes][kV * NC] then inclusive values [32 lanes][kV * NS].
-template <class Map, int NS>
+// Descriptor of one tile (or group of tiles) in the workspace, in tagged
+// words: aggregates [32 lanes][kV * NC], then inclusive values
+// [32 lanes][kV * NS].  Agg = false drops the aggregates, for look-backs that
+// only ever wait for inclusive values: the descriptors are then a third
+// (ParaGRU) or a quarter (ParaLSTM) as large, and so is their zeroing.
+template <class Map, int NS, bool Agg = true>
 struct TileDesc {
-    static constexpr int agg_words = 32 * kV * Map::kFloats;
-    static constexpr int words = 32 * kV * (Map::kFloats + NS);
+    static constexpr int agg_words = Agg ? 32 * kV * Map::kFloats : 0;
+    static constexpr int words = agg_words + 32 * kV * NS;
 };
 
 // Store n (even) tagged words.
@@ -93,22 +96,22 @@ struct LookbackProbe {
 
 // (WithAgg = false: the inclusive value only, for a look-back that waits for
 // it instead of stepping back.)
-template <class Map, int NS, bool WithAgg = true>
+template <class Map, int NS, bool WithAgg = true, class TD = TileDesc<Map, NS>>
 __device__ __forceinline__ void lookback_probe(LookbackProbe<Map, NS>& pr, int pred_ticket,
                                                const unsigned long long* desc, int lane)
 {
-    using TD = TileDesc<Map, NS>;
+    static_assert(!WithAgg || TD::agg_words > 0, "descriptors without aggregates");
     const unsigned long long* pd = desc + (size_t)pred_ticket * TD::words;
     load_words(pd + TD::agg_words + lane * kV * NS, pr.wi);
     if (WithAgg) load_words(pd + lane * kV * Map::kFloats, pr.wa);
 }
 
 // Publish maps (a tile's or a group's aggregate) under tag 2*epoch+1.
-template <class Map, int NS>
+template <class Map, int NS, class TD = TileDesc<Map, NS>>
 __device__ __forceinline__ void publish_aggregate(unsigned long long* desc, int ticket, int epoch, const Map (&ta)[kV],
                                                   int lane)
 {
-    using TD = TileDesc<Map, NS>;
+    static_assert(TD::agg_words > 0, "descriptors without aggregates");
     constexpr int NC = Map::kFloats;
     float av[kV * NC];
 #pragma unroll
@@ -120,11 +123,10 @@ __device__ __forceinline__ void publish_aggregate(unsigned long long* desc, int 
 
 // Publish an inclusive value (the state leaving a tile or group) under tag
 // 2*epoch+2.
-template <class Map, int NS>
+template <class Map, int NS, class TD = TileDesc<Map, NS>>
 __device__ __forceinline__ void publish_inclusive(unsigned long long* desc, int ticket, int epoch,
                                                   const float (&incl)[NS][kV], int lane)
 {
-    using TD = TileDesc<Map, NS>;
     float iv[kV * NS];
 #pragma unroll
     for (int j = 0; j < kV; ++j)
@@ -145,10 +147,11 @@ __device__ __forceinline__ void publish_inclusive(unsigned long long* desc, int 
 //              values, which is faster when few tiles of one sequence are in
 //              flight at once) and read no aggregates at all (the probe must
 //              then come from lookback_probe<..., false>)
+//   TD:        the descriptor layout (aggregate-free only when !Walk)
 // Each step back reads the predecessor's inclusive value and aggregate
 // together (one round trip).  Each lane walks back on its own; a wait that
 // runs out of time raises PARARNN_ERR_TIMEOUT and returns false.
-template <class Map, int NS, bool Walk = true>
+template <class Map, int NS, bool Walk = true, class TD = TileDesc<Map, NS>>
 __device__ __forceinline__ bool lookback_resolve(int ticket, int stride, int epoch, float (&carry)[NS][kV],
                                                  const unsigned long long* desc, int lane, int* err,
                                                  unsigned long long wait_ns, LookbackProbe<Map, NS>& pr)
@@ -188,7 +191,7 @@ __device__ __forceinline__ bool lookback_resolve(int ticket, int stride, int epo
                 }
                 jt -= stride;
                 spins = 0;
-                lookback_probe(pr, jt, desc, lane);
+                lookback_probe<Map, NS, Walk, TD>(pr, jt, desc, lane);  // (Walk is true here)
             } else {
                 // predecessor not published yet: back off, bounded
                 if ((++spins & 15u) == 0u) {
@@ -207,7 +210,7 @@ __device__ __forceinline__ bool lookback_resolve(int ticket, int stride, int epo
                     }
                 }
                 if (spins > 32) __nanosleep(64);
-                if (!done) lookback_probe<Map, NS, Walk>(pr, jt, desc, lane);
+                if (!done) lookback_probe<Map, NS, Walk, TD>(pr, jt, desc, lane);
             }
         }
     }

@@ -94,3 +94,30 @@ def test_lstm_training_step_fullsize_sampled(cuda):
         assert H.max_abs(duc[:, :, :, d].double().numpy(), rdu[:, :, :, 0]) <= 1e-4 * scale
         bound = 1e-5 * np.sum(np.abs(rdu[:, :, :, 0]), axis=(0, 1)) + 1e-6
         assert np.all(np.abs(dac[:, d].double().numpy() - rda[:, 0]) <= bound)
+
+
+def test_gru_training_step_fullsize_sampled(cuda):
+    w = W.GRU_TRAIN
+    x = W.make_inputs(w, seed=0)
+    xd = x.to(cuda)
+    pk = P()
+    h, it, r, st = pk.pararnn_gru_solve(xd.u, xd.a, xd.h0, tol=w.tol, max_iters=w.max_iters)
+    du, da, dh0 = pk.pararnn_gru_adjoint(xd.u, xd.a, xd.h0, h, xd.dh)
+    torch.cuda.synchronize()
+    assert st == 0
+    assert bool(torch.isfinite(du).all()) and bool(torch.isfinite(da).all())
+    rng = np.random.default_rng(6)
+    ds = sorted({0, w.D - 1, *[int(v) for v in rng.integers(0, w.D, 4)]})
+    duc, dac, dh0c = du.cpu(), da.cpu(), dh0.cpu()
+    for d in ds:
+        # all batches of channel d (da sums over b and l)
+        u = H.f64(x.u[:, :, :, d:d + 1])
+        a = H.f64(x.a[:, d:d + 1])
+        h0 = H.f64(x.h0[:, d:d + 1])
+        gh = H.f64(x.dh[:, :, d:d + 1])
+        rdu, rda, rdh0 = oracle.gru_bptt(u, a, h0, gh)
+        scale = max(1.0, float(np.abs(rdu).max()))
+        assert H.max_abs(duc[:, :, :, d].double().numpy(), rdu[:, :, :, 0]) <= 1e-4 * scale
+        assert H.max_abs(dh0c[:, d].double().numpy(), rdh0[:, 0]) <= 1e-4 * scale
+        bound = 1e-5 * np.sum(np.abs(rdu[:, :, :, 0]), axis=(0, 1)) + 1e-6
+        assert np.all(np.abs(dac[:, d].double().numpy() - rda[:, 0]) <= bound)
