@@ -17,11 +17,9 @@
 // (d pre / d a) du over b and l in a fixed order (deterministic), and the
 // gradient of the initial state is mu_1.
 //
-// This header holds what the scan kernel shares with the host: its
-// parameter block and the fixed-order reduction of da.
+// This header holds the scan kernel's parameter block; the fixed-order
+// reduction of da is in da_reduce.cuh.
 #pragma once
-
-#include <climits>
 
 #include "scan_common.cuh"
 
@@ -41,34 +39,5 @@ struct AdjointParams {
     float* partial;       // [B][n_chunks][S][G][kDc] per-tile sums for da
     unsigned long long wait_ns;
 };
-
-// da[g][d] = sum over b, then chunk c, of the per-tile partial sums, in a
-// fixed order.  Block: 32 columns x 8 row-groups; each row-group sums every
-// 8th (b, c) row, the 8 group sums are then added in group order.
-__global__ void __launch_bounds__(256) da_reduce_kernel(const float* __restrict__ partial, float* __restrict__ da,
-                                                        int rows /* B*n_chunks */, int S, int G, long long D)
-{
-    __shared__ float red[8][33];
-    const int col = blockIdx.x * 32 + (threadIdx.x & 31);  // index over G*D
-    const int grp = threadIdx.x >> 5;
-    const long long GD = (long long)G * D;
-    float acc = 0.f;
-    int g = 0, s = 0, dd = 0;
-    if (col < GD) {
-        g = int(col / D);
-        const long long d = col - (long long)g * D;
-        s = int(d / kDc);
-        dd = int(d - (long long)s * kDc);
-        for (int r = grp; r < rows; r += 8) acc += partial[(((size_t)r * S + s) * G + g) * kDc + dd];
-    }
-    red[grp][threadIdx.x & 31] = acc;
-    __syncthreads();
-    if (grp == 0 && col < GD) {
-        float t = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t += red[i][threadIdx.x];
-        da[col] = t;
-    }
-}
 
 }  // namespace pararnn

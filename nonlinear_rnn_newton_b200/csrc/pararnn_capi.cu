@@ -23,6 +23,7 @@
 #include "decode.cuh"
 #include "segment.cuh"
 #include "adjoint.cuh"
+#include "da_reduce.cuh"
 #include "selftest.cuh"
 #include "adjoint_ws.cuh"
 #include "linear_scan.cuh"
@@ -737,6 +738,39 @@ template <class Cell, class UT> constexpr int adj_warps()
 // workspace sizing uses the shortest tile (most tiles) of either gate dtype
 template <class Cell> constexpr int adj_lc_min() { return 2 * adj_warps<Cell, float>(); }
 
+// Row slabs of the da reduction: about 1024 blocks of da_slab_kernel, and no
+// more slabs than rows.  A function of the shape alone, so that the sums are
+// added in the same order on every run.
+int da_slabs(long long rows, int S, int G)
+{
+    const long long SG = (long long)S * G;
+    return int(std::max(1LL, std::min(rows, (1024 + SG - 1) / SG)));
+}
+
+// Workspace bytes after the descriptors: the per-tile partial sums
+// [B*n_chunks][S][G][kDc], then the slab sums [slabs][S][G][kDc].
+size_t da_bytes(const Shape& s, int G)
+{
+    const long long rows = s.B * s.n_chunks;
+    return (size_t(s.n_tiles) + size_t(da_slabs(rows, s.S, G)) * s.S) * G * kDc * 4;
+}
+
+// da from the partial sums (`partial` at the start of the da_bytes region).
+pararnn_status da_reduce(float* partial, float* da, const Shape& s, int G, cudaStream_t stream)
+{
+    const long long rows = s.B * s.n_chunks;
+    const int slabs = da_slabs(rows, s.S, G);
+    float* sums = partial + size_t(s.n_tiles) * G * kDc;
+    da_slab_kernel<<<dim3(unsigned(s.S * G), unsigned(slabs)), kDc, 0, stream>>>(partial, sums, int(rows), slabs,
+                                                                                 s.S * G);
+    CUDA_TRY(cudaGetLastError());
+    const long long GD = (long long)G * s.D;
+    da_final_kernel<<<unsigned((GD + 255) / 256), 256, 0, stream>>>(sums, da, slabs, s.S, G, s.D);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(2, std::memory_order_relaxed);
+    return PARARNN_OK;
+}
+
 size_t adjoint_ws_bytes(int cell, long long B, long long L, long long D)
 {
     if (!shape_ok(B, L, D) || D % 8 != 0) return 0;
@@ -748,7 +782,7 @@ size_t adjoint_ws_bytes(int cell, long long B, long long L, long long D)
     if (st != PARARNN_OK) return 0;
     const int G = cell == 0 ? 3 : 4;
     const int desc = cell == 0 ? TileDesc<Aff<1>, 1, false>::words : TileDesc<Aff<2>, 2, false>::words;
-    return scan_layout(s, desc, size_t(s.n_tiles) * G * kDc * 4).total;
+    return scan_layout(s, desc, da_bytes(s, G)).total;
 }
 
 template <class Cell, class UT>
@@ -760,7 +794,7 @@ pararnn_status launch_adjoint(Shape s, const void* u, pararnn_dtype dt, const fl
     using LY = AdjointWsLayout<Cell, UT, CW>;
     constexpr int NS = Cell::NS, G = Cell::G;
     TRY(make_shape(s.B, s.L, s.D, LY::Lc, &s));
-    const ScanLayout ly = scan_layout(s, LY::desc_words, size_t(s.n_tiles) * G * kDc * 4);
+    const ScanLayout ly = scan_layout(s, LY::desc_words, da_bytes(s, G));
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     CUDA_TRY(cudaMemsetAsync(ws, 0, ly.extra, stream));
 
@@ -799,11 +833,8 @@ pararnn_status launch_adjoint(Shape s, const void* u, pararnn_dtype dt, const fl
     TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid, LY::threads));
     kern<<<grid, LY::threads, LY::smem_bytes, stream>>>(tu, t0, t1, tg0, tg1, p);
     CUDA_TRY(cudaGetLastError());
-    const long long GD = (long long)G * s.D;
-    da_reduce_kernel<<<unsigned((GD + 31) / 32), 256, 0, stream>>>(p.partial, da, int(s.B) * s.n_chunks, s.S, G, s.D);
-    CUDA_TRY(cudaGetLastError());
-    g_launches.fetch_add(2, std::memory_order_relaxed);
-    return PARARNN_OK;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return da_reduce(p.partial, da, s, G, stream);
 }
 
 pararnn_status adjoint_async(int cell, const void* u, pararnn_dtype dt, const float* a, const float* c0,
