@@ -19,7 +19,7 @@
 //     turns the folds into exclusive prefixes (latest steps first), takes
 //     the carry from the later tile's published value, and writes it.
 // After sweep 2 the compute warps add their da partials of the tile in warp
-// order (a named barrier among them), so that da is reproducible.
+// order (between two named barriers among them), so that da is reproducible.
 #pragma once
 
 #include <climits>
@@ -48,13 +48,14 @@ struct AdjointWsLayout {
     static constexpr size_t g_bytes = a128(g_tx);
     static constexpr size_t stage_bytes = off_g + NS * g_bytes;
     // work buffer: folds, then exclusive prefixes [NC][CW][kDc] | carry [NS][kDc]
-    // | da partials of the compute warps [CW][G][kDc]
     static constexpr size_t off_agg = 0;
     static constexpr size_t off_carry = a128(size_t(NC) * CW * kDc * 4);
-    static constexpr size_t off_dacc = off_carry + a128(size_t(NS) * kDc * 4);
-    static constexpr size_t work_bytes = off_dacc + a128(size_t(CW) * G * kDc * 4);
+    static constexpr size_t work_bytes = off_carry + a128(size_t(NS) * kDc * 4);
     static constexpr size_t off_work = kStages * stage_bytes;
-    static constexpr size_t off_misc = off_work + kWork * work_bytes;
+    // the da partials of the compute warps [CW][G][kDc], one buffer: every
+    // tile's are added up between two barriers of the compute warps
+    static constexpr size_t off_dacc = off_work + kWork * work_bytes;
+    static constexpr size_t off_misc = off_dacc + a128(size_t(CW) * G * kDc * 4);
     // misc: full, empty per stage; aggr, carry per work buffer; a job
     // (ticket, chunk, batch row, first channel) per stage; flags
     static constexpr size_t misc_bytes = a128((2 * kStages + 2 * kWork) * 8 + kStages * 16 + 8 * 4);
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 }
                 // the tile's da partial: every warp's sums in shared memory,
                 // then each warp adds up a slice of them in warp order
-                float* sd = reinterpret_cast<float*>(work_at(wp) + LY::off_dacc);
+                float* sd = reinterpret_cast<float*>(smem + LY::off_dacc);
 #pragma unroll
                 for (int g = 0; g < G; ++g) store4(sd + (w * G + g) * kDc + lane * kV, dacc[g]);
                 compute_sync();
@@ -419,6 +420,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     for (int ww = 0; ww < CW; ++ww) acc += sd[ww * G * kDc + i];
                     part[i] = acc;
                 }
+                compute_sync();  // the buffer is free for the next tile's partials
             }
             if (!valid) break;
             prev = job;

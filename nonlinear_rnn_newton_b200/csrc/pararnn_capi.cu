@@ -726,10 +726,10 @@ pararnn_status project_solve_async(const void* x, const void* w, const float* bi
 // gate dtype; fp32 gates need twice the staging space, so their tiles are half
 // as long.
 #ifndef PARARNN_ADJ_GRU_WARPS
-#define PARARNN_ADJ_GRU_WARPS 14
+#define PARARNN_ADJ_GRU_WARPS 15
 #endif
 #ifndef PARARNN_ADJ_LSTM_WARPS
-#define PARARNN_ADJ_LSTM_WARPS 7
+#define PARARNN_ADJ_LSTM_WARPS 8
 #endif
 template <class Cell, class UT> constexpr int adj_warps()
 {
