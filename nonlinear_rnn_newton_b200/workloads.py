@@ -56,11 +56,13 @@ LSTM_TRAIN = Workload("lstm_train_bf16_B4_L16384_D2048", "lstm", 4, 16384, 2048,
 GRU_TRAIN = Workload("gru_train_bf16_B4_L16384_D2048", "gru", 4, 16384, 2048, "bf16", h0_std=0.1,
                      train=True)
 
-# the training workload at L/4 and D/2 (an eighth of its elements): ~0.6 GB
-# on the device, still larger than L2 -- a size a full profiler capture of
-# the adjoint handles
+# the training workloads at L/4 and D/2 (an eighth of their elements): about
+# 0.5 GB on the device, still larger than L2 -- a size a full profiler
+# capture of the adjoint handles
 LSTM_TRAIN_SMALL = Workload("lstm_train_bf16_B4_L4096_D1024", "lstm", 4, 4096, 1024, "bf16", train=True)
-ALL = (GRU_SMALL, GRU, LSTM) + GRU_SWEEP + (LSTM_TRAIN, GRU_TRAIN, LSTM_TRAIN_SMALL)
+GRU_TRAIN_SMALL = Workload("gru_train_bf16_B4_L4096_D1024", "gru", 4, 4096, 1024, "bf16", h0_std=0.1,
+                           train=True)
+ALL = (GRU_SMALL, GRU, LSTM) + GRU_SWEEP + (LSTM_TRAIN, GRU_TRAIN, LSTM_TRAIN_SMALL, GRU_TRAIN_SMALL)
 BY_NAME = {w.name: w for w in ALL}
 
 
