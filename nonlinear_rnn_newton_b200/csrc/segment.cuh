@@ -97,14 +97,19 @@ __host__ __device__ inline long long fold_steps(long long Ls)
 // zero guess) composed in order into part [nf][NC][B][D], and max |F| of the
 // steps into *res.  Page: "A sacada: método de Newton" (the Newton step is the
 // linear recurrence s^{k+1}_l = J_l s^{k+1}_{l-1} + o_l, o_l = f_l - J_l s^k_{l-1}).
+// A step's map needs only H^k, so two consecutive steps are evaluated
+// together in the packed two-row form of the cell (channel pairs in float2,
+// reciprocals shared between the rows), as in the fused pass.
 template <class Cell, class UT>
 __global__ void __launch_bounds__(128) segment_fold_kernel(const UT* __restrict__ u, const float* __restrict__ a,
                                                            const float* __restrict__ s_in, float* __restrict__ part,
                                                            unsigned* res, long long B, long long Ls, long long D,
                                                            int steps)
 {
-    using Map = typename Cell::Map;
-    constexpr int G = Cell::G, NS = Cell::NS, NC = Map::kFloats;
+    using Packed = typename Cell::Packed;
+    using Map2 = typename Packed::Map2;
+    using Rows2 = typename Packed::Rows2;
+    constexpr int G = Cell::G, NS = Cell::NS, NC = Cell::Map::kFloats, NP = kV / 2;
     const long long D4 = D >> 2, BD = B * D, per = B * Ls * D;
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     float rmax = 0.f;
@@ -112,64 +117,117 @@ __global__ void __launch_bounds__(128) segment_fold_kernel(const UT* __restrict_
         const long long b = i / D4, d = (i - b * D4) << 2;
         const long long l0 = 1 + (long long)blockIdx.y * steps;
         const long long l1 = l0 + steps < Ls ? l0 + steps : Ls;
-        float av[G][kV];
+        float2 av[G][NP];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             const F4 x = load4(a + g * D + d);
 #pragma unroll
-            for (int j = 0; j < kV; ++j) av[g][j] = x.v[j];
+            for (int jp = 0; jp < NP; ++jp) av[g][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
         }
-        float prev[NS][kV];
+        // gates and H^k of step l, as channel pairs
+        auto load_step = [&](long long l, float2 (&ug)[G][NP], float2 (&hk)[NS][NP]) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const F4 x = load4(u + ((b * Ls + l) * G + g) * D + d);
+#pragma unroll
+                for (int jp = 0; jp < NP; ++jp) ug[g][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
+            }
+#pragma unroll
+            for (int q = 0; q < NS; ++q) {
+                F4 x{{0.f, 0.f, 0.f, 0.f}};
+                if (s_in) x = load4(s_in + q * per + (b * Ls + l) * D + d);
+#pragma unroll
+                for (int jp = 0; jp < NP; ++jp) hk[q][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
+            }
+        };
+        auto keep_max = [&](float2 h, float2 f) {
+            rmax = max_nan(rmax, fabsf(h.x - f.x));
+            rmax = max_nan(rmax, fabsf(h.y - f.y));
+        };
+        // H^k before the first step
+        float2 prev[NS][NP];
 #pragma unroll
         for (int q = 0; q < NS; ++q) {
             F4 x{{0.f, 0.f, 0.f, 0.f}};
             if (s_in) x = load4(s_in + q * per + (b * Ls + l0 - 1) * D + d);
 #pragma unroll
-            for (int j = 0; j < kV; ++j) prev[q][j] = x.v[j];
+            for (int jp = 0; jp < NP; ++jp) prev[q][jp] = make_float2(x.v[2 * jp], x.v[2 * jp + 1]);
         }
-        Map acc[kV];
+        Map2 acc[NP];
 #pragma unroll
-        for (int j = 0; j < kV; ++j) acc[j] = Map::identity();
-        // unrolled so that the loads of several steps are in flight together
-#pragma unroll 4
-        for (long long l = l0; l < l1; ++l) {
-            F4 ug[G], cur[NS];
+        for (int jp = 0; jp < NP; ++jp) acc[jp] = Map2::identity();
+        long long l = l0;
+        // (both steps' loads are in flight together; unrolling further measured
+        // slower, from the registers it takes)
+#pragma unroll 1
+        for (; l + 1 < l1; l += 2) {
+            float2 ua[G][NP], ub[G][NP], ha[NS][NP], hb[NS][NP];
+            load_step(l, ua, ha);
+            load_step(l + 1, ub, hb);
 #pragma unroll
-            for (int g = 0; g < G; ++g) ug[g] = load4(u + ((b * Ls + l) * G + g) * D + d);
-#pragma unroll
-            for (int q = 0; q < NS; ++q) {
-                cur[q] = F4{{0.f, 0.f, 0.f, 0.f}};
-                if (s_in) cur[q] = load4(s_in + q * per + (b * Ls + l) * D + d);
-            }
-#pragma unroll
-            for (int j = 0; j < kV; ++j) {
-                float sp[NS], uu[G], aa[G], f[NS], js[NS];
-#pragma unroll
-                for (int q = 0; q < NS; ++q) sp[q] = prev[q][j];
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    uu[g] = ug[g].v[j];
-                    aa[g] = av[g][j];
-                }
-                Map m;
-                Cell::eval(sp, uu, aa, f, m);
-                apply_matrix(m, sp, js);
-                float o[NS];
+            for (int jp = 0; jp < NP; ++jp) {
+                float2 sa[NS], sb[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS], ja[NS], jb[NS], oa[NS], ob[NS];
 #pragma unroll
                 for (int q = 0; q < NS; ++q) {
-                    o[q] = f[q] - js[q];
-                    rmax = max_nan(rmax, fabsf(cur[q].v[j] - f[q]));
-                    prev[q][j] = cur[q].v[j];
+                    sa[q] = prev[q][jp];
+                    sb[q] = ha[q][jp];
                 }
-                set_map_offset(m, o);
-                acc[j] = compose(m, acc[j]);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    u_a[g] = ua[g][jp];
+                    u_b[g] = ub[g][jp];
+                    aa[g] = av[g][jp];
+                }
+                Map2 ea, eb;
+                Rows2::eval(sa, u_a, sb, u_b, aa, fa, fb, ea, eb);
+                apply_matrix2(ea, sa, ja);
+                apply_matrix2(eb, sb, jb);
+#pragma unroll
+                for (int q = 0; q < NS; ++q) {
+                    oa[q] = fma2(ja[q], bc2(-1.0f), fa[q]);
+                    ob[q] = fma2(jb[q], bc2(-1.0f), fb[q]);
+                    keep_max(ha[q][jp], fa[q]);
+                    keep_max(hb[q][jp], fb[q]);
+                    prev[q][jp] = hb[q][jp];
+                }
+                set_offset2(ea, oa);
+                set_offset2(eb, ob);
+                acc[jp] = compose(eb, compose(ea, acc[jp]));
+            }
+        }
+        if (l < l1) {  // an odd step left
+            float2 ua[G][NP], ha[NS][NP];
+            load_step(l, ua, ha);
+#pragma unroll
+            for (int jp = 0; jp < NP; ++jp) {
+                float2 sa[NS], u_a[G], aa[G], fa[NS], ja[NS], oa[NS];
+#pragma unroll
+                for (int q = 0; q < NS; ++q) sa[q] = prev[q][jp];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    u_a[g] = ua[g][jp];
+                    aa[g] = av[g][jp];
+                }
+                Map2 ea;
+                Packed::eval(sa, u_a, aa, fa, ea);
+                apply_matrix2(ea, sa, ja);
+#pragma unroll
+                for (int q = 0; q < NS; ++q) {
+                    oa[q] = fma2(ja[q], bc2(-1.0f), fa[q]);
+                    keep_max(ha[q][jp], fa[q]);
+                }
+                set_offset2(ea, oa);
+                acc[jp] = compose(ea, acc[jp]);
             }
         }
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             float v[kV];
 #pragma unroll
-            for (int j = 0; j < kV; ++j) v[j] = acc[j].get(c);
+            for (int jp = 0; jp < NP; ++jp) {
+                v[2 * jp] = acc[jp].lane(0).get(c);
+                v[2 * jp + 1] = acc[jp].lane(1).get(c);
+            }
             store4(part + ((long long)blockIdx.y * NC + c) * BD + b * D + d, v);
         }
     }
