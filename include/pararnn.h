@@ -422,7 +422,8 @@ PARARNN_API pararnn_status pararnn_lstm_segment_pass(const void* u, pararnn_dtyp
  * entries, NS = 1 or 2, G = 3 or 4), then 4 floats (the first is the
  * residual over the segment's steps 2..Ls).  0 for invalid arguments. */
 PARARNN_API size_t pararnn_segment_record_floats(int n_state, int64_t B, int64_t D);
-/* Workspace bytes of segment_fold (its per-128-step partial folds). */
+/* Workspace bytes of segment_fold (its partial folds, one per part of 64 or
+ * more steps). */
 PARARNN_API size_t pararnn_segment_fold_workspace_size(int n_state, int64_t B, int64_t L, int64_t D);
 /* segment_fold: the segment's record (overwritten in full) from the iterate
  * s_in [NS][B][Ls][D] (NULL = the zero guess) and the gates u [B][Ls][G][D]
