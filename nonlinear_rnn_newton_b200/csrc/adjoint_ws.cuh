@@ -28,10 +28,14 @@
 
 namespace pararnn {
 
-template <class Cell, class UT, int CW>
+// NG: upstream gradient components staged per tile -- NS, or 1 when only the
+// last component (h) has one (a ParaLSTM loss on h alone), which leaves room
+// for more compute warps.
+template <class Cell, class UT, int CW, int NG = Cell::NS>
 struct AdjointWsLayout {
     static constexpr int G = Cell::G;
     static constexpr int NS = Cell::NS;
+    static_assert(NG == NS || NG == 1, "staged upstream components");
     static constexpr int NC = Cell::Map::kFloats;
     static constexpr int Lc = 2 * CW;
     static constexpr int kStages = 3;
@@ -40,13 +44,15 @@ struct AdjointWsLayout {
     static constexpr size_t u_tx = size_t(Lc) * G * kDc * sizeof(UT);
     static constexpr size_t s_tx = size_t(Lc + 1) * kDc * 4;  // states from the row before the tile
     static constexpr size_t g_tx = size_t(Lc) * kDc * 4;
-    // ring stage: gates | states [NS] | upstream [NS]
+    // ring stage: gates | states [NS] | upstream [NG]
     static constexpr size_t off_u = 0;
     static constexpr size_t off_s = a128(u_tx);
     static constexpr size_t s_bytes = a128(s_tx);
     static constexpr size_t off_g = off_s + NS * s_bytes;
     static constexpr size_t g_bytes = a128(g_tx);
-    static constexpr size_t stage_bytes = off_g + NS * g_bytes;
+    static constexpr size_t stage_bytes = off_g + NG * g_bytes;
+    // the upstream slot of component q (with NG = 1 only the last one is staged)
+    static constexpr int g_slot(int q) { return NG == NS ? q : 0; }
     // work buffer: folds, then exclusive prefixes [NC][CW][kDc] | carry [NS][kDc]
     static constexpr size_t off_agg = 0;
     static constexpr size_t off_carry = a128(size_t(NC) * CW * kDc * 4);
@@ -73,16 +79,19 @@ __device__ __forceinline__ void compute_sync_n()
     asm volatile("bar.sync 1, %0;" ::"n"(32 * CW) : "memory");
 }
 
-template <class Cell, class UT, int CW>
+template <class Cell, class UT, int CW, int NG = Cell::NS>
 __global__ void __launch_bounds__(32 * (CW + 1), 1)
     adjoint_ws_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_s0,
                       const __grid_constant__ CUtensorMap tm_s1, const __grid_constant__ CUtensorMap tm_g0,
                       const __grid_constant__ CUtensorMap tm_g1, const AdjointParams p)
 {
-    using LY = AdjointWsLayout<Cell, UT, CW>;
+    using LY = AdjointWsLayout<Cell, UT, CW, NG>;
     using Map = typename Cell::Map;
     using TD = TileDesc<Map, Cell::NS, false>;  // inclusive values only
     constexpr int G = LY::G, NS = LY::NS, NC = LY::NC, Lc = LY::Lc;
+    // upstream gradient of component q present and staged (with NG = 1 the
+    // host launches this kernel only when component 0 has none)
+    auto staged = [&](int q) { return p.has_g[q] != 0 && (NG == NS || q == NS - 1); };
     constexpr int kStages = LY::kStages, kWork = LY::kWork;
     static_assert(LY::fits, "shared memory");
 
@@ -133,15 +142,15 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 uint32_t bytes = uint32_t(LY::u_tx + NS * LY::s_tx);
 #pragma unroll
                 for (int q = 0; q < NS; ++q)
-                    if (p.has_g[q]) bytes += uint32_t(LY::g_tx);
+                    if (staged(q)) bytes += uint32_t(LY::g_tx);
                 mbar_arrive_expect_tx(&bar_full[stage], bytes);
                 tma_load_4d(st + LY::off_u, &tm_u, d0, 0, c * Lc, b, &bar_full[stage]);
                 // rows c*Lc - 1 .. c*Lc + Lc - 1 (the row before the first chunk reads as zeros)
                 tma_load_3d(st + LY::off_s, &tm_s0, d0, c * Lc - 1, b, &bar_full[stage]);
                 if (NS == 2) tma_load_3d(st + LY::off_s + LY::s_bytes, &tm_s1, d0, c * Lc - 1, b, &bar_full[stage]);
-                if (p.has_g[0]) tma_load_3d(st + LY::off_g, &tm_g0, d0, c * Lc, b, &bar_full[stage]);
-                if (NS == 2 && p.has_g[1])
-                    tma_load_3d(st + LY::off_g + LY::g_bytes, &tm_g1, d0, c * Lc, b, &bar_full[stage]);
+                if (staged(0)) tma_load_3d(st + LY::off_g, &tm_g0, d0, c * Lc, b, &bar_full[stage]);
+                if (NS == 2 && staged(1))
+                    tma_load_3d(st + LY::off_g + LY::g_slot(1) * LY::g_bytes, &tm_g1, d0, c * Lc, b, &bar_full[stage]);
             } else {
                 s_job[stage] = make_int4(INT_MAX, 0, 0, 0);
                 mbar_arrive(&bar_full[stage]);
@@ -259,7 +268,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                         if (chv && p.s0[q]) x = load4(p.s0[q] + b * D + dch);
                     }
                     F4 z{{0.f, 0.f, 0.f, 0.f}};
-                    if (p.has_g[q]) z = load4(sg + q * (LY::g_bytes / 4) + row * kDc + lane * kV);
+                    if (staged(q)) z = load4(sg + LY::g_slot(q) * (LY::g_bytes / 4) + row * kDc + lane * kV);
 #pragma unroll
                     for (int j = 0; j < kV; ++j) {
                         sv[q][j] = x.v[j];

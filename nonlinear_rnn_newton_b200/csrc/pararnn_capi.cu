@@ -722,21 +722,30 @@ pararnn_status project_solve_async(const void* x, const void* w, const float* bi
 
 // --------------------------------------------------------------- adjoints
 
-// Compute warps (two steps each) of the warp-specialised adjoint per cell and
-// gate dtype; fp32 gates need twice the staging space, so their tiles are half
-// as long.
+// Compute warps (two steps each) of the warp-specialised adjoint per cell,
+// gate dtype and staged upstream components (NG; a ParaLSTM loss on h alone
+// stages one, which leaves shared memory for a ninth warp); fp32 gates need
+// twice the staging space, so their tiles are half as long.
 #ifndef PARARNN_ADJ_GRU_WARPS
 #define PARARNN_ADJ_GRU_WARPS 15
 #endif
 #ifndef PARARNN_ADJ_LSTM_WARPS
 #define PARARNN_ADJ_LSTM_WARPS 8
 #endif
-template <class Cell, class UT> constexpr int adj_warps()
+#ifndef PARARNN_ADJ_LSTM_H_WARPS
+#define PARARNN_ADJ_LSTM_H_WARPS 9
+#endif
+template <class Cell, class UT, int NG> constexpr int adj_warps()
 {
-    return (Cell::NS == 1 ? PARARNN_ADJ_GRU_WARPS : PARARNN_ADJ_LSTM_WARPS) / (sizeof(UT) == 2 ? 1 : 2);
+    return (Cell::NS == 1 ? PARARNN_ADJ_GRU_WARPS : NG == 1 ? PARARNN_ADJ_LSTM_H_WARPS : PARARNN_ADJ_LSTM_WARPS) /
+           (sizeof(UT) == 2 ? 1 : 2);
 }
-// workspace sizing uses the shortest tile (most tiles) of either gate dtype
-template <class Cell> constexpr int adj_lc_min() { return 2 * adj_warps<Cell, float>(); }
+// workspace sizing uses the shortest tile (most tiles) of any variant
+template <class Cell> constexpr int adj_lc_min()
+{
+    constexpr int a = adj_warps<Cell, float, Cell::NS>(), b = adj_warps<Cell, float, 1>();
+    return 2 * (a < b ? a : b);
+}
 
 // Row slabs of the da reduction: about 1024 blocks of da_slab_kernel, and no
 // more slabs than rows.  A function of the shape alone, so that the sums are
@@ -785,13 +794,13 @@ size_t adjoint_ws_bytes(int cell, long long B, long long L, long long D)
     return scan_layout(s, desc, da_bytes(s, G)).total;
 }
 
-template <class Cell, class UT>
+template <class Cell, class UT, int NG = Cell::NS>
 pararnn_status launch_adjoint(Shape s, const void* u, pararnn_dtype dt, const float* a, const float* const s0[2],
                               const float* const st[2], const float* const g[2], float* du, float* da,
                               float* const ds0[2], void* ws, cudaStream_t stream)
 {
-    constexpr int CW = adj_warps<Cell, UT>();
-    using LY = AdjointWsLayout<Cell, UT, CW>;
+    constexpr int CW = adj_warps<Cell, UT, NG>();
+    using LY = AdjointWsLayout<Cell, UT, CW, NG>;
     constexpr int NS = Cell::NS, G = Cell::G;
     TRY(make_shape(s.B, s.L, s.D, LY::Lc, &s));
     const ScanLayout ly = scan_layout(s, LY::desc_words, da_bytes(s, G));
@@ -828,7 +837,7 @@ pararnn_status launch_adjoint(Shape s, const void* u, pararnn_dtype dt, const fl
     p.partial = reinterpret_cast<float*>(wsb + ly.extra);
     p.wait_ns = kWaitLimitNs;
 
-    auto kern = adjoint_ws_kernel<Cell, UT, CW>;
+    auto kern = adjoint_ws_kernel<Cell, UT, CW, NG>;
     int grid = 0;
     TRY(resident_grid(kern, LY::smem_bytes, s.n_tiles, &grid, LY::threads));
     kern<<<grid, LY::threads, LY::smem_bytes, stream>>>(tu, t0, t1, tg0, tg1, p);
@@ -874,6 +883,11 @@ pararnn_status adjoint_async(int cell, const void* u, pararnn_dtype dt, const fl
     const float* st[2] = {c, h};
     const float* g[2] = {dc, dh};
     float* ds0[2] = {dc0, dh0};
+    if (!dc) {  // a loss on h alone: one upstream component staged
+        if (dt == PARARNN_BF16)
+            return launch_adjoint<LstmCell, uint16_t, 1>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+        return launch_adjoint<LstmCell, float, 1>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
+    }
     if (dt == PARARNN_BF16)
         return launch_adjoint<LstmCell, uint16_t>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
     return launch_adjoint<LstmCell, float>(s, u, dt, a, s0, st, g, du, da, ds0, ws, stream);
