@@ -101,6 +101,12 @@ struct NewtonWsLayout {
     static constexpr bool fits = smem_bytes <= 232448;  // opt-in shared memory per CTA
 };
 
+// both halves finite (NaN and inf fail the comparison)
+__device__ __forceinline__ bool finite2(float2 v)
+{
+    return fabsf(v.x) <= 3.40282347e38f && fabsf(v.y) <= 3.40282347e38f;
+}
+
 // Seg: the segment-pass form (warm start and a separate linearisation point
 // for chunk 0, read from the workspace header); a template parameter so that
 // the plain solve keeps its own code.
@@ -180,6 +186,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 // slot (k+1)%3 was last used two passes ago; every CTA is past it
                 hdr->tick[(k + 1) % 3] = 0u;
                 hdr->res[(k + 1) % 3] = 0u;
+                hdr->over[(k + 1) % 3] = 0u;
             }
             // fresh barriers every pass (no copy is in flight between passes)
             for (int i = 0; i < kStages; ++i) {
@@ -455,6 +462,11 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 (void)mbar_wait_bounded(&bar_full[s], uint32_t(n / kStages) & 1u, err, p.wait_ns);
                 const int4 job = s_job[s];
                 const bool valid = job.x < p.n_tiles;
+                // whether a tile of this pass has found a residual above tol
+                // (read now, used in sweep 2 below: the load is in flight
+                // during sweep 1)
+                const int over_seen =
+                    (NS == 1 && lane == 0) ? ld_relaxed_gpu(reinterpret_cast<const int*>(&hdr->over[slot])) : 0;
                 Jac2 Jn[2][NP];
                 if (valid) {
                     // ---- sweep 1 of tile n
@@ -639,6 +651,15 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             for (int q = 0; q < NS; ++q) y0[q][jp] = z[q];
                         }
                     }
+                    // (ParaGRU) Once a tile of this pass has found a residual
+                    // above tol, the pass cannot end the solve with its
+                    // residual reported (only a pass whose residual is <= tol,
+                    // or the last allowed one, does), so the rest of its tiles
+                    // leave the residual out -- unless a new state is not
+                    // finite, which decides the outcome, and then the tile
+                    // evaluates it.  Every decision stays the same; only the
+                    // maxima of passes that continue are partial.
+                    const bool skip_ok = NS == 1 && k + 1 < p.max_iters && __shfl_sync(0xffffffffu, over_seen, 0) != 0;
                     float2 offa[NS][NP], offb[NS][NP], ua[G][NP], ub[G][NP];
 #pragma unroll
                     for (int q = 0; q < NS; ++q) {
@@ -663,32 +684,92 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     const long long la = l0 + ra, lb = l0 + rb;
                     const bool va = la < L && chv, vb = lb < L && chv;
                     float2 ya[NS][NP], yb[NS][NP];
+                    if constexpr (NS == 1) {
 #pragma unroll
-                    for (int jp = 0; jp < NP; ++jp) {
-                        float2 s0v[NS], sav[NS], sbv[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS], t0[NS], t1[NS];
+                        for (int jp = 0; jp < NP; ++jp) {
+                            float2 s0v[NS], sav[NS], t0[NS], t1[NS];
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) s0v[q] = y0[q][jp];
-                        apply_matrix2(Jp[0][jp], s0v, t0);
+                            for (int q = 0; q < NS; ++q) s0v[q] = y0[q][jp];
+                            apply_matrix2(Jp[0][jp], s0v, t0);
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) sav[q] = add2(t0[q], offa[q][jp]);
-                        apply_matrix2(Jp[1][jp], sav, t1);
+                            for (int q = 0; q < NS; ++q) sav[q] = add2(t0[q], offa[q][jp]);
+                            apply_matrix2(Jp[1][jp], sav, t1);
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) sbv[q] = add2(t1[q], offb[q][jp]);
-#pragma unroll
-                        for (int g = 0; g < G; ++g) {
-                            u_a[g] = ua[g][jp];
-                            u_b[g] = ub[g][jp];
-                            aa[g] = wv[g][jp];
+                            for (int q = 0; q < NS; ++q) {
+                                ya[q][jp] = sav[q];
+                                yb[q][jp] = add2(t1[q], offb[q][jp]);
+                            }
                         }
-                        Rows2::value(s0v, u_a, sav, u_b, aa, fa, fb);
+                        bool eval = !skip_ok;
+                        if (skip_ok) {
+                            bool finite = true;
 #pragma unroll
-                        for (int q = 0; q < NS; ++q) {
-                            const float2 da = add2(sav[q], neg2(fa[q]));
-                            const float2 db = add2(sbv[q], neg2(fb[q]));
-                            if (va) rpost = max_keep_nan(rpost, max_keep_nan(fabsf(da.x), fabsf(da.y)));
-                            if (vb) rpost = max_keep_nan(rpost, max_keep_nan(fabsf(db.x), fabsf(db.y)));
-                            ya[q][jp] = sav[q];
-                            yb[q][jp] = sbv[q];
+                            for (int jp = 0; jp < NP; ++jp)
+#pragma unroll
+                                for (int q = 0; q < NS; ++q) {
+                                    if (va) finite = finite && finite2(ya[q][jp]);
+                                    if (vb) finite = finite && finite2(yb[q][jp]);
+                                }
+                            eval = !__all_sync(0xffffffffu, finite);
+                        }
+                        if (eval) {
+                            float tmax = 0.f;
+#pragma unroll
+                            for (int jp = 0; jp < NP; ++jp) {
+                                float2 s0v[NS], sav[NS], sbv[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS];
+#pragma unroll
+                                for (int q = 0; q < NS; ++q) {
+                                    s0v[q] = y0[q][jp];
+                                    sav[q] = ya[q][jp];
+                                    sbv[q] = yb[q][jp];
+                                }
+#pragma unroll
+                                for (int g = 0; g < G; ++g) {
+                                    u_a[g] = ua[g][jp];
+                                    u_b[g] = ub[g][jp];
+                                    aa[g] = wv[g][jp];
+                                }
+                                Rows2::value(s0v, u_a, sav, u_b, aa, fa, fb);
+#pragma unroll
+                                for (int q = 0; q < NS; ++q) {
+                                    const float2 da = add2(sav[q], neg2(fa[q]));
+                                    const float2 db = add2(sbv[q], neg2(fb[q]));
+                                    if (va) tmax = max_keep_nan(tmax, max_keep_nan(fabsf(da.x), fabsf(da.y)));
+                                    if (vb) tmax = max_keep_nan(tmax, max_keep_nan(fabsf(db.x), fabsf(db.y)));
+                                }
+                            }
+                            rpost = max_keep_nan(rpost, tmax);
+                            const bool above = !(tmax <= p.tol);  // NaN counts
+                            if (__any_sync(0xffffffffu, above) && !skip_ok && lane == 0) atomicMax(&hdr->over[slot], 1u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) {
+                            float2 s0v[NS], sav[NS], sbv[NS], u_a[G], u_b[G], aa[G], fa[NS], fb[NS], t0[NS], t1[NS];
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) s0v[q] = y0[q][jp];
+                            apply_matrix2(Jp[0][jp], s0v, t0);
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) sav[q] = add2(t0[q], offa[q][jp]);
+                            apply_matrix2(Jp[1][jp], sav, t1);
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) sbv[q] = add2(t1[q], offb[q][jp]);
+#pragma unroll
+                            for (int g = 0; g < G; ++g) {
+                                u_a[g] = ua[g][jp];
+                                u_b[g] = ub[g][jp];
+                                aa[g] = wv[g][jp];
+                            }
+                            Rows2::value(s0v, u_a, sav, u_b, aa, fa, fb);
+#pragma unroll
+                            for (int q = 0; q < NS; ++q) {
+                                const float2 da = add2(sav[q], neg2(fa[q]));
+                                const float2 db = add2(sbv[q], neg2(fb[q]));
+                                if (va) rpost = max_keep_nan(rpost, max_keep_nan(fabsf(da.x), fabsf(da.y)));
+                                if (vb) rpost = max_keep_nan(rpost, max_keep_nan(fabsf(db.x), fabsf(db.y)));
+                                ya[q][jp] = sav[q];
+                                yb[q][jp] = sbv[q];
+                            }
                         }
                     }
 #pragma unroll

@@ -41,7 +41,10 @@ struct alignas(256) WsHeader {
     // projection kernel (which then left H^1, the residuals of H^0 and H^1
     // in res0 and res[0], and its own ticket count in tick[3]).
     int k0;
-    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result) - 8 * kPassTimes - 8 * 2 - 4 - 4];
+    // Per pass slot: a tile of the pass has found a residual above tol (or
+    // NaN), so the pass cannot end the solve with its residual reported.
+    unsigned over[4];
+    unsigned char pad[256 - 4 * 4 * 2 - 4 * 4 - sizeof(pararnn_result) - 8 * kPassTimes - 8 * 2 - 4 - 4 - 4 * 4];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
 
