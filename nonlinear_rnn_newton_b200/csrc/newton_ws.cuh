@@ -655,7 +655,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     // above tol, the pass cannot end the solve with its
                     // residual reported (only a pass whose residual is <= tol,
                     // or the last allowed one, does), so the rest of its tiles
-                    // leave the residual out -- unless a new state is not
+                    // leave the residual out -- unless a state it reads is not
                     // finite, which decides the outcome, and then the tile
                     // evaluates it.  Every decision stays the same; only the
                     // maxima of passes that continue are partial.
@@ -707,7 +707,9 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             for (int jp = 0; jp < NP; ++jp)
 #pragma unroll
                                 for (int q = 0; q < NS; ++q) {
-                                    if (va) finite = finite && finite2(ya[q][jp]);
+                                    // (the state entering the warp's steps too:
+                                    // a residual reads the state before its step)
+                                    if (va) finite = finite && finite2(y0[q][jp]) && finite2(ya[q][jp]);
                                     if (vb) finite = finite && finite2(yb[q][jp]);
                                 }
                             eval = !__all_sync(0xffffffffu, finite);

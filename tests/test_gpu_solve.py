@@ -179,6 +179,43 @@ def test_nonfinite_input_reports_nonfinite(cuda):
     assert st == -5
 
 
+def _same_outcome(a, b):
+    """(states, iters, residual, status) equal, NaN where NaN."""
+    (ha, ia, ra, sa), (hb, ib, rb, sb) = a, b
+    assert (ia, sa) == (ib, sb)
+    assert (math.isnan(ra) and math.isnan(rb)) or ra == rb
+    assert np.array_equal(np.isnan(ha), np.isnan(hb))
+    assert np.array_equal(np.nan_to_num(ha), np.nan_to_num(hb))
+
+
+@pytest.mark.parametrize("shape", [(8, 4096, 1024), (1, 8192, 2048)], ids=["B8", "B1"])
+def test_partial_residuals_leave_the_outcome_unchanged(cuda, shape):
+    """A ParaGRU pass that is not the last allowed one stops evaluating the
+    residual once a tile has found one above tol.  The same solve capped at
+    its own iteration count (every pass then evaluates it in full, the last
+    one being the last allowed) must give the same states, count, residual
+    and status."""
+    B, L, D = shape
+    w = W.custom("gru", B, L, D, "bf16", h0_std=0.1)
+    x = W.make_inputs(w, seed=21)
+    full = run_gru(x, cuda, max_iters=10)
+    assert full[3] == 0 and full[1] >= 3
+    capped = run_gru(x, cuda, max_iters=full[1])
+    _same_outcome(full, capped)
+
+
+def test_iterates_that_overflow_report_nonfinite(cuda):
+    """Recurrence weights so large that the Newton update overflows: the
+    non-finite states must be caught in the pass that makes them, as when
+    that pass is the last allowed one (full residual)."""
+    w = W.custom("gru", 2, 3000, 256, "bf16", h0_std=0.1)
+    x = W.make_inputs(w, seed=22, a_scale=4000.0)
+    out = run_gru(x, cuda, max_iters=10)
+    assert out[3] == -5 and not np.isfinite(out[0]).all()
+    capped = run_gru(x, cuda, max_iters=out[1])
+    _same_outcome(out, capped)
+
+
 def test_solve_is_deterministic(cuda):
     w = W.custom("gru", 4, 2048, 512, "bf16", h0_std=0.1)
     x = W.make_inputs(w, seed=14).to(cuda)
