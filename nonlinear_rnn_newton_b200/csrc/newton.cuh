@@ -35,6 +35,7 @@ struct NewtonParams {
     float* bnd;             // [2][NS][B][n_chunks][S*kDc]
     unsigned long long wait_ns;
     int lb_walk;            // look-backs step over aggregates (many groups of a sequence in flight)
+    int skip_res;           // ParaGRU: passes that continue may leave residuals out (many tiles per CTA)
 };
 
 

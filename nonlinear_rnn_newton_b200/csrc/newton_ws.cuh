@@ -465,6 +465,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 // whether a tile of this pass has found a residual above tol
                 // (read now, used in sweep 2 below: the load is in flight
                 // during sweep 1)
+                // (never set where p.skip_res is 0)
                 const int over_seen =
                     (NS == 1 && lane == 0) ? ld_relaxed_gpu(reinterpret_cast<const int*>(&hdr->over[slot])) : 0;
                 Jac2 Jn[2][NP];
@@ -742,7 +743,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             }
                             rpost = max_keep_nan(rpost, tmax);
                             const bool above = !(tmax <= p.tol);  // NaN counts
-                            if (__any_sync(0xffffffffu, above) && !skip_ok && lane == 0) atomicMax(&hdr->over[slot], 1u);
+                            if (p.skip_res && __any_sync(0xffffffffu, above) && !skip_ok && lane == 0)
+                                atomicMax(&hdr->over[slot], 1u);
                         }
                     } else {
 #pragma unroll

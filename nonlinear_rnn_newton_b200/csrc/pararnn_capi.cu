@@ -135,6 +135,13 @@ long long solve_descs(const Shape& s) { return solve_desc_count(s.n_chunks, s.B 
 // L=65536 D=2048: 2.81 against 3.17 ms).
 int solve_lookback_walks(int grid, long long sequences) { return grid >= 4 * sequences ? 1 : 0; }
 
+// Whether ParaGRU passes that continue may leave residuals out once a tile has
+// found one above tol.  It pays where each CTA runs several tiles a pass; with
+// about one or two (short sequences) the flag arrives too late to spare much
+// and its checks cost more than they save (measured at B1 D2048: L = 512
+// 0.0615 ms without, 0.065 with; L = 2048 0.137 with, 0.141 without).
+int solve_skips_residuals(long long n_tiles, int grid) { return n_tiles >= 4LL * grid ? 1 : 0; }
+
 size_t solve_bnd_bytes(const Shape& s, int NS)
 {
     return size_t(2) * NS * s.B * s.n_chunks * s.S * kDc * 4;
@@ -346,6 +353,7 @@ pararnn_status launch_newton_k(const Shape& s, const void* u, pararnn_dtype dt, 
     int grid = 0;
     TRY(resident_grid(kern, KL::smem_bytes, s.n_tiles, &grid, threads));
     p.lb_walk = LB;
+    p.skip_res = solve_skips_residuals(s.n_tiles, grid);
     CUtensorMap ta, tb;
     TRY(map_weights(&ta, a, Cell::G, s));
     TRY(map_bnd(&tb, p.bnd, NS, s));
