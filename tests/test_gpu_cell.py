@@ -119,6 +119,22 @@ def test_max_iters_and_tol_rules(cuda, compiled):
     assert it == 1 and H.max_abs(s.cpu(), H1) <= TOL_STATE
 
 
+@pytest.mark.parametrize("fast", [0, 1])
+def test_partial_residuals_leave_a_user_cell_outcome_unchanged(cuda, compiled, fast):
+    """A one-component user cell on enough tiles that passes which continue
+    leave residuals out: the solve capped at its own iteration count (every
+    pass evaluating the residual in full) gives the same states, count,
+    residual and status."""
+    cell = CELLS["gru"]
+    u, a, s0 = draw(cell, 8, 2048, 512, "bf16", seed=9)
+    ud, ad, sd = u.to(cuda), a.to(cuda), s0.to(cuda)
+    s1, it1, r1, st1 = P().pararnn_cell_solve(compiled["gru", fast], ud, ad, sd, max_iters=10)
+    assert st1 == 0 and it1 >= 3
+    s2, it2, r2, st2 = P().pararnn_cell_solve(compiled["gru", fast], ud, ad, sd, max_iters=it1)
+    assert (it2, st2, r2) == (it1, st1, r1)
+    assert torch.equal(s1, s2)
+
+
 ADJ_SHAPES = [(2, 300, 136, "bf16"), (3, 257, 64, "f32"), (1, 1, 8, "bf16")]
 
 
