@@ -216,4 +216,17 @@ struct GenericCell {
     };
 };
 
+// A two-component user cell in accurate math leaves residuals out in the
+// passes that continue (its residual evaluation, with the library's accurate
+// functions, is a large share of a pass); with the fast functions it keeps
+// the full evaluation, as the built-in ParaLSTM does.
+template <int G_>
+struct PartialResiduals<GenericCell<G_, 2>> {
+#ifdef PARARNN_USER_FAST_MATH
+    static constexpr bool value = false;
+#else
+    static constexpr bool value = true;
+#endif
+};
+
 }  // namespace pararnn

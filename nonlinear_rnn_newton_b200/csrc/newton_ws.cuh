@@ -101,6 +101,14 @@ struct NewtonWsLayout {
     static constexpr bool fits = smem_bytes <= 232448;  // opt-in shared memory per CTA
 };
 
+// Whether passes that continue may leave residuals out (see sweep 2): the
+// one-component cells; a two-component cell's own specialisation may opt in
+// (the built-in ParaLSTM measured no faster with it).
+template <class Cell>
+struct PartialResiduals {
+    static constexpr bool value = Cell::NS == 1;
+};
+
 // both halves finite (NaN and inf fail the comparison)
 __device__ __forceinline__ bool finite2(float2 v)
 {
@@ -466,8 +474,9 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                 // (read now, used in sweep 2 below: the load is in flight
                 // during sweep 1)
                 // (never set where p.skip_res is 0)
-                const int over_seen =
-                    (NS == 1 && lane == 0) ? ld_relaxed_gpu(reinterpret_cast<const int*>(&hdr->over[slot])) : 0;
+                const int over_seen = (PartialResiduals<Cell>::value && lane == 0)
+                                          ? ld_relaxed_gpu(reinterpret_cast<const int*>(&hdr->over[slot]))
+                                          : 0;
                 Jac2 Jn[2][NP];
                 if (valid) {
                     // ---- sweep 1 of tile n
@@ -652,7 +661,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                             for (int q = 0; q < NS; ++q) y0[q][jp] = z[q];
                         }
                     }
-                    // (ParaGRU) Once a tile of this pass has found a residual
+                    // (PartialResiduals) Once a tile of this pass has found a residual
                     // above tol, the pass cannot end the solve with its
                     // residual reported (only a pass whose residual is <= tol,
                     // or the last allowed one, does), so the rest of its tiles
@@ -660,7 +669,8 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     // finite, which decides the outcome, and then the tile
                     // evaluates it.  Every decision stays the same; only the
                     // maxima of passes that continue are partial.
-                    const bool skip_ok = NS == 1 && k + 1 < p.max_iters && __shfl_sync(0xffffffffu, over_seen, 0) != 0;
+                    const bool skip_ok = PartialResiduals<Cell>::value && k + 1 < p.max_iters &&
+                                         __shfl_sync(0xffffffffu, over_seen, 0) != 0;
                     float2 offa[NS][NP], offb[NS][NP], ua[G][NP], ub[G][NP];
 #pragma unroll
                     for (int q = 0; q < NS; ++q) {
@@ -685,7 +695,7 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1)
                     const long long la = l0 + ra, lb = l0 + rb;
                     const bool va = la < L && chv, vb = lb < L && chv;
                     float2 ya[NS][NP], yb[NS][NP];
-                    if constexpr (NS == 1) {
+                    if constexpr (PartialResiduals<Cell>::value) {
 #pragma unroll
                         for (int jp = 0; jp < NP; ++jp) {
                             float2 s0v[NS], sav[NS], t0[NS], t1[NS];
